@@ -1,0 +1,351 @@
+"""Checks that pin the CPU oracle to things other than itself.
+
+Each ``check_*`` takes an oracle instance and raises AssertionError if the
+oracle disagrees with what the paper's method and the mathematics fix:
+hand-worked fixtures under ``tests/golden/``, library routines (numpy's
+float32 division and rint, numpy's int64 matmul, torch's bf16 rounding),
+exact rational arithmetic, closed forms and invariants.  The same checks
+are run against deliberately broken copies of the oracle to show that a
+plausible mistake anywhere in it fails at least one of them.
+
+Method: "Realizing Native INT8 Compute for Diffusion Transformers on
+Consumer GPUs" (arXiv 2606.14598), abstract -- per-token activation
+quantization, per-channel weight quantization, int8 x int8 -> int32 GEMM,
+per-token x per-channel dequantization plus bias in the epilogue, bf16 out.
+"""
+from __future__ import annotations
+
+import os
+from fractions import Fraction
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+U32 = 2.0 ** -24   # binary32 unit roundoff
+U16 = 2.0 ** -8    # bf16 unit roundoff (8 significant bits)
+
+
+# ------------------------------------------------------------- helpers
+
+
+def bf16_bits(values) -> np.ndarray:
+    """Exact bf16 bit patterns of values that torch can represent exactly."""
+    t = torch.tensor(np.asarray(values, np.float32)).to(torch.bfloat16)
+    assert (t.float().numpy() == np.asarray(values, np.float32)).all(), "value not exact in bf16"
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def bits_to_float(bits) -> np.ndarray:
+    t = torch.from_numpy(np.asarray(bits, np.uint16).view(np.int16).copy()).view(torch.bfloat16)
+    return t.float().numpy()
+
+
+def read_rows(name: str):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as fh:
+        for line in fh:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            parts = [p.split() for p in line.split("|")]
+            rows.append(parts)
+    return rows
+
+
+def parse_num(tok: str) -> float:
+    """A decimal, or a*2^b for exact powers of two (e.g. subnormals)."""
+    if "*2^" in tok:
+        a, b = tok.split("*2^")
+        return float(a) * 2.0 ** int(b)
+    return float(tok)
+
+
+def read_keyed(name: str) -> dict:
+    out: dict = {}
+    with open(os.path.join(GOLDEN, name)) as fh:
+        for line in fh:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *vals = line.split()
+            out.setdefault(key, []).append([float(v) for v in vals])
+    return out
+
+
+def numpy_quantize(x: np.ndarray):
+    """The quantizer through numpy's float32 routines (library cross-check)."""
+    x = x.astype(np.float32)
+    amax = np.max(np.abs(x), axis=1)
+    s = (amax / np.float32(127.0)).astype(np.float32)
+    q = np.zeros(x.shape, np.int8)
+    nz = amax > 0
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = (x[nz] / s[nz, None]).astype(np.float32)
+    q[nz] = np.clip(np.rint(t), -127, 127).astype(np.int8)
+    return q, s
+
+
+def edge_rows(K: int, rng: np.random.Generator) -> np.ndarray:
+    """bf16 rows that exercise the quantizer's special cases."""
+    rows = []
+    z = np.zeros(K, np.float32)
+    rows.append(z.copy())                                  # all zero
+    r = z.copy(); r[K // 3] = -3.0; rows.append(r)         # single non-zero, negative
+    r = -z; rows.append(r)                                 # all -0
+    r = rng.standard_normal(K).astype(np.float32) * np.float32(2.0 ** -130); rows.append(r)  # subnormal
+    r = np.full(K, 0.5, np.float32); r[0] = 127.0; rows.append(r)          # ties at .5
+    r = (np.arange(K, dtype=np.float32) % 255 - 127) + np.float32(0.5)    # many ties
+    r[1] = 127.0; rows.append(np.clip(r, -127, 127))
+    r = rng.standard_normal(K).astype(np.float32) * np.float32(1e4); rows.append(r)  # large
+    return bits_to_float(torch.tensor(np.stack(rows)).to(torch.bfloat16).view(torch.int16).numpy()
+                         .view(np.uint16))
+
+
+def to_bits(x: np.ndarray) -> np.ndarray:
+    return torch.tensor(np.asarray(x, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+# ------------------------------------------------------------- bf16
+
+
+def check_bf16_widen(orc) -> None:
+    """bf16 -> f32 equals torch's conversion on every non-NaN bit pattern."""
+    pats = np.arange(0, 65536, dtype=np.uint32).astype(np.uint16)
+    mine = orc.bf16_bits_to_f32(pats)
+    ref = bits_to_float(pats)
+    ok = np.isnan(ref) | (mine.view(np.uint32) == ref.view(np.uint32))
+    assert ok.all(), "bf16 widening differs from torch"
+
+
+def check_bf16_round(orc) -> None:
+    """f32 -> bf16 RNE equals torch's conversion, ties and overflow included."""
+    rng = np.random.default_rng(11)
+    hi = rng.integers(0, 65536, 4000).astype(np.uint32) << 16
+    lows = np.array([0, 1, 0x7fff, 0x8000, 0x8001, 0xffff], np.uint32)
+    u = (hi[:, None] | lows[None, :]).reshape(-1)
+    f = u.view(np.float32)
+    f = f[~np.isnan(f)]
+    extra = np.array([3.3895314e38, 3.4028235e38, -3.4028235e38, 1e-45, -0.0, 0.0, np.inf, -np.inf],
+                     np.float32)
+    f = np.concatenate([f, extra])
+    mine = orc.f32_to_bf16_bits(f)
+    ref = torch.from_numpy(f.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert (mine == ref).all(), f"bf16 rounding differs from torch at {np.flatnonzero(mine != ref)[:5]}"
+
+
+# ------------------------------------------------------------ quantizer
+
+
+def check_quant_golden(orc) -> None:
+    """Hand-worked rows (tests/golden/quant_act_rows.txt)."""
+    for xs, qs, ss in read_rows("quant_act_rows.txt"):
+        x = np.array([float(v) for v in xs], np.float32)
+        q, s = orc.quantize_act(bf16_bits(x)[None, :])
+        want = np.array([int(v) for v in qs], np.int8)
+        assert (q[0] == want).all(), f"codes {q[0]} != {want} for {x}"
+        if ss[0] != "-":
+            assert s[0] == np.float32(float(ss[0])), f"scale {s[0]} != {ss[0]}"
+
+
+def check_weight_golden(orc) -> None:
+    """Hand-worked fp32 weight rows (tests/golden/quant_weight_rows.txt)."""
+    for ws, qs, ss in read_rows("quant_weight_rows.txt"):
+        w = np.array([parse_num(v) for v in ws], np.float32)
+        assert (w.astype(np.float64) == np.array([parse_num(v) for v in ws])).all(), "not exact in fp32"
+        q, s = orc.quantize_weight(w[None, :])
+        assert (q[0] == np.array([int(v) for v in qs], np.int8)).all(), f"codes {q[0]} for {w}"
+        assert s[0] == np.float32(parse_num(ss[0]))
+
+
+def check_quant_vs_numpy(orc) -> None:
+    """Quantizer equals the same rule through numpy float32 division + rint."""
+    rng = np.random.default_rng(5)
+    K = 200
+    x = np.concatenate([edge_rows(K, rng),
+                        bits_to_float(to_bits(rng.standard_normal((40, K)).astype(np.float32)))])
+    q, s = orc.quantize_act(to_bits(x))
+    q2, s2 = numpy_quantize(x)
+    assert (s.view(np.uint32) == s2.view(np.uint32)).all(), "scales differ from numpy"
+    assert (q == q2).all(), "codes differ from numpy"
+    w = rng.standard_normal((30, 96)).astype(np.float32) * np.float32(0.02)
+    wq, sw = orc.quantize_weight(w)
+    wq2, sw2 = numpy_quantize(w)
+    assert (sw.view(np.uint32) == sw2.view(np.uint32)).all() and (wq == wq2).all()
+
+
+def check_quant_invariants(orc) -> None:
+    """Properties any per-token absmax quantizer with round-to-nearest has."""
+    rng = np.random.default_rng(6)
+    K = 300
+    x = bits_to_float(to_bits(rng.standard_normal((64, K)).astype(np.float32)
+                              * np.float32(3.0) ** rng.integers(-3, 4, (64, 1)).astype(np.float32)))
+    q, s = orc.quantize_act(to_bits(x))
+    amax = np.abs(x).max(axis=1)
+    # the largest |x| of every row maps to +-127 with the sign of x
+    arg = np.abs(x).argmax(axis=1)
+    assert (np.abs(q).max(axis=1) == 127).all()
+    assert (q[np.arange(64), arg] == np.sign(x[np.arange(64), arg]) * 127).all()
+    # round to nearest: |q*s - x| <= s/2 (plus the rounding of s and of x/s)
+    err = np.abs(q.astype(np.float64) * s[:, None].astype(np.float64) - x.astype(np.float64))
+    assert (err <= s[:, None] * (0.5 + 1e-4)).all(), "reconstruction error above half a step"
+    # scale s is absmax/127 to within one binary32 rounding
+    assert np.allclose(s.astype(np.float64), amax.astype(np.float64) / 127.0, rtol=2 * U32, atol=0)
+    # exact power-of-two scaling: same codes, scale times 2^j
+    for j in (-5, 7):
+        q2, s2 = orc.quantize_act(to_bits(x * np.float32(2.0 ** j)))
+        assert (q2 == q).all() and (s2 == s * np.float32(2.0 ** j)).all()
+    # negation: codes negate, scale unchanged
+    q3, s3 = orc.quantize_act(to_bits(-x))
+    assert (q3 == -q).all() and (s3 == s).all()
+    # row independence: permuting tokens permutes results
+    perm = rng.permutation(64)
+    q4, s4 = orc.quantize_act(to_bits(x[perm]))
+    assert (q4 == q[perm]).all() and (s4 == s[perm]).all()
+
+
+# ----------------------------------------------------------------- GEMM
+
+
+def check_gemm_vs_numpy(orc) -> None:
+    """Exact accumulator equals numpy's int64 matmul (and a Python brute force)."""
+    rng = np.random.default_rng(7)
+    for M, N, K in [(1, 1, 1), (5, 3, 7), (33, 17, 96), (70, 40, 272)]:
+        a = rng.integers(-127, 128, (M, K), dtype=np.int8)
+        b = rng.integers(-127, 128, (N, K), dtype=np.int8)
+        acc = orc.gemm_i64(a, b, nthreads=3)
+        assert (acc == a.astype(np.int64) @ b.astype(np.int64).T).all()
+    a = rng.integers(-127, 128, (3, 5), dtype=np.int8)
+    b = rng.integers(-127, 128, (4, 5), dtype=np.int8)
+    acc = orc.gemm_i64(a, b)
+    for m in range(3):
+        for n in range(4):
+            assert acc[m, n] == sum(int(a[m, k]) * int(b[n, k]) for k in range(5))
+
+
+def check_gemm_closed_forms(orc) -> None:
+    """Identity and one-hot weights; worst-case all-+-127 rows at K = 12288."""
+    rng = np.random.default_rng(8)
+    K = 48
+    xq = rng.integers(-127, 128, (9, K), dtype=np.int8)
+    eye = (np.eye(K, dtype=np.int64) * 127).astype(np.int8)
+    assert (orc.gemm_i64(xq, eye) == 127 * xq.astype(np.int64)).all()
+    cols = rng.integers(0, K, 20)
+    onehot = np.zeros((20, K), np.int8)
+    onehot[np.arange(20), cols] = 1
+    assert (orc.gemm_i64(xq, onehot) == xq[:, cols].astype(np.int64)).all()
+    K = 12288
+    x = np.stack([np.full(K, 127, np.int8), np.full(K, -127, np.int8)])
+    acc = orc.gemm_i64(x, x)
+    big = K * 127 * 127
+    assert big == 198193152 and big < 2 ** 31
+    assert (acc == np.array([[big, -big], [-big, big]])).all()
+
+
+def check_gemm_invariants(orc) -> None:
+    rng = np.random.default_rng(9)
+    a = rng.integers(-127, 128, (12, 64), dtype=np.int8)
+    b = rng.integers(-127, 128, (10, 64), dtype=np.int8)
+    acc = orc.gemm_i64(a, b)
+    pm, pn = rng.permutation(12), rng.permutation(10)
+    assert (orc.gemm_i64(a[pm], b[pn]) == acc[pm][:, pn]).all()
+    assert (orc.gemm_i64(-a, b) == -acc).all()
+    pk = rng.permutation(64)   # permuting the reduction index changes nothing
+    assert (orc.gemm_i64(a[:, pk], b[:, pk]) == acc).all()
+
+
+# ------------------------------------------------------------- epilogue
+
+
+def _exact_y(acc, sa, sw, bias_f) -> list:
+    return [[Fraction(int(acc[m, n])) * Fraction(float(sa[m])) * Fraction(float(sw[n]))
+             + Fraction(float(bias_f[n])) for n in range(acc.shape[1])] for m in range(acc.shape[0])]
+
+
+def check_epilogue_exact_bound(orc) -> None:
+    """bf16 output within the binary32 + bf16 rounding bound of the exact value."""
+    rng = np.random.default_rng(10)
+    M, N = 24, 20
+    acc = rng.integers(-200_000_000, 200_000_000, (M, N)).astype(np.int64)
+    acc[0, :] = 0
+    sa = np.exp(rng.uniform(np.log(1e-4), np.log(1e-1), M)).astype(np.float32)
+    sw = np.exp(rng.uniform(np.log(1e-4), np.log(1e-1), N)).astype(np.float32)
+    bias = to_bits(rng.standard_normal(N).astype(np.float32) * np.float32(0.1))
+    bias_f = bits_to_float(bias)
+    out = bits_to_float(orc.epilogue(acc, sa, sw, bias))
+    y = _exact_y(acc, sa, sw, bias_f)
+    for m in range(M):
+        for n in range(N):
+            prod = abs(float(Fraction(int(acc[m, n])) * Fraction(float(sa[m])) * Fraction(float(sw[n]))))
+            ye = float(y[m][n])
+            bound = U16 * abs(ye) + 4 * U32 * (prod + abs(float(bias_f[n]))) + 1e-38
+            assert abs(float(out[m, n]) - ye) <= bound, (m, n, out[m, n], ye)
+    # a zero accumulator gives the bias exactly
+    assert (out[0] == bias_f).all()
+    # the fp64 recomputation agrees with the exact value to binary64 precision
+    y64 = orc.epilogue_f64(acc, sa, sw, bias)
+    for m in range(M):
+        for n in range(N):
+            assert abs(y64[m, n] - float(y[m][n])) <= 4 * 2.0 ** -53 * (abs(float(y[m][n])) + 1.0)
+
+
+def check_epilogue_bias_optional(orc) -> None:
+    rng = np.random.default_rng(12)
+    acc = rng.integers(-10 ** 6, 10 ** 6, (5, 8)).astype(np.int64)
+    sa = np.full(5, 0.01, np.float32)
+    sw = np.full(8, 0.02, np.float32)
+    zero = np.zeros(8, np.uint16)
+    assert (orc.epilogue(acc, sa, sw, None) == orc.epilogue(acc, sa, sw, zero)).all()
+
+
+def check_hand_linear(orc) -> None:
+    """The worked example of tests/golden/hand_linear_2x4x2.txt, step by step."""
+    g = read_keyed("hand_linear_2x4x2.txt")
+    x = bf16_bits(np.array(g["x"], np.float32))
+    wq = np.array(g["wq"], np.int8)
+    sw = np.array(g["scale_w"][0], np.float32)
+    bias = bf16_bits(np.array(g["bias"][0], np.float32))
+    out, xq, sa, acc = orc.linear(x, wq, sw, bias)
+    assert (xq == np.array(g["xq"], np.int8)).all()
+    assert (sa == np.array(g["scale_a"][0], np.float32)).all()
+    assert (acc == np.array(g["acc"], np.int64)).all()
+    assert (bits_to_float(out) == np.array(g["out"], np.float32)).all(), bits_to_float(out)
+
+
+def check_linear_identity_weight(orc) -> None:
+    """Identity weight (127 * I, scale 1/127), zero bias: out ~ X within the
+    quantization step of each token."""
+    rng = np.random.default_rng(13)
+    K = 64
+    x = to_bits(rng.standard_normal((16, K)).astype(np.float32))
+    xf = bits_to_float(x).astype(np.float64)
+    wq = (np.eye(K) * 127).astype(np.int8)
+    sw = np.full(K, np.float32(1.0) / np.float32(127.0), np.float32)
+    out, xq, sa, acc = orc.linear(x, wq, sw, np.zeros(K, np.uint16))
+    y = bits_to_float(out).astype(np.float64)
+    step = sa.astype(np.float64)[:, None]
+    assert (np.abs(y - xf) <= 0.5 * step * (1 + 1e-3) + U16 * np.abs(xf) + 1e-30).all()
+
+
+def check_linear_composition(orc) -> None:
+    """The whole layer equals its three steps run one after another."""
+    rng = np.random.default_rng(14)
+    x = to_bits(rng.standard_normal((20, 80)).astype(np.float32))
+    wq = rng.integers(-127, 128, (24, 80), dtype=np.int8)
+    sw = np.exp(rng.uniform(-9, -2, 24)).astype(np.float32)
+    bias = to_bits(rng.standard_normal(24).astype(np.float32))
+    out, xq, sa, acc = orc.linear(x, wq, sw, bias)
+    q2, s2 = orc.quantize_act(x)
+    a2 = orc.gemm_i64(q2, wq)
+    assert (q2 == xq).all() and (s2 == sa).all() and (a2 == acc).all()
+    assert (orc.epilogue(a2, s2, sw, bias) == out).all()
+
+
+ALL_CHECKS = [
+    check_bf16_widen, check_bf16_round,
+    check_quant_golden, check_weight_golden, check_quant_vs_numpy, check_quant_invariants,
+    check_gemm_vs_numpy, check_gemm_closed_forms, check_gemm_invariants,
+    check_epilogue_exact_bound, check_epilogue_bias_optional,
+    check_hand_linear, check_linear_identity_weight, check_linear_composition,
+]
