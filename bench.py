@@ -1,0 +1,460 @@
+"""Benchmark of the W8A8 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl native|reference]
+
+One step is one W8A8 linear layer (per-token quantization -> tcgen05 int8
+GEMM -> dequant + bias epilogue -> bf16) over one token batch of the
+workload, by default the 1024px DiT MLP up-projection (M=4096 tokens,
+K=3072, N=12288).  Inputs are seeded synthetic data resident in HBM; the
+step cycles through enough buffer sets (activations, weights, workspace,
+output) that their combined footprint is several times the 126 MB L2, so
+every step reads its operands from HBM.
+
+Printed (rank 0, one JSON line): whole-job int8 TOPS (2*M*N*K per step,
+summed over ranks, divided by the max over ranks of the device time),
+the GEMM kernel's roofline against the int8 tensor peak, the quantizer's
+GB/s, the end-to-end figure through the public API with host buffers, the
+CPU oracle timed on a bounded sample, SM clocks sampled during the timed
+region, and context (bf16 torch.matmul and the dequantize-then-bf16-GEMM
+path on the same shape).
+
+Multi-GPU (torchrun, one process per GPU): tokens are independent, so each
+rank runs its own token batch against a replicated weight with no
+data-path collective (weak scaling); torch.distributed is used only for the
+barrier and the max over ranks of the timed region.
+
+--impl reference times the CPU oracle (the plain C reference of the method)
+on the host cores instead, on a bounded row sample per step, and prints
+the same metric for it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "fused W8A8 linear TOPS and % of B200 dense INT8 peak per M×N×K; quantizer GB/s"
+L2_BYTES = 126 * 1024 * 1024
+NOMINAL_INT8_OVER_BF16 = 2.0     # 4.5 POPS dense int8 / 2.25 PFLOP/s dense bf16 (B200 datasheet)
+SPEC_INT8_POPS = 4500.0          # B200 dense int8, TOPS
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+GEMM_SOURCES = ["w8a8_int8_gemm_b200/csrc/gemm_sm100.cu", "w8a8_int8_gemm_b200/csrc/sm100_ptx.cuh",
+                "w8a8_int8_gemm_b200/csrc/api.cu"]
+
+
+# ---------------------------------------------------------------- helpers
+
+
+def dist_env() -> tuple[int, int, int]:
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def gemm_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str) -> dict | None:
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
+    taken on the current GEMM sources (else None)."""
+    path = os.path.join(ROOT, "profiles", f"gemm_{workload}_dram.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+    except (OSError, ValueError):
+        return None
+    if d.get("gemm_source_hash") != gemm_source_hash():
+        return None
+    return d
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during a region."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", sel, f"--query-gpu={','.join(self.FIELDS)}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, RuntimeError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(", ") for r in out.strip().splitlines() if r.count(",") >= len(self.FIELDS) - 1]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        pw = [float(r[2]) for r in rows if r[2].replace(".", "", 1).isdigit()]
+        loaded = [s for s, p in zip(sm, pw) if p > 300] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None,
+                "samples": len(rows), "reasons": reasons}
+
+
+# ------------------------------------------------------------ CPU oracle
+
+
+class OracleWork:
+    """The workload prepared once for the CPU oracle: the weight quantized by
+    the oracle, and a pool of token rows.  sample(rows, cols, i) runs the
+    whole layer (quantize, exact GEMM, epilogue) for `rows` tokens against
+    the first `cols` output channels and returns its wall time."""
+
+    def __init__(self, wl: workloads.Workload, pool_rows: int = 512):
+        import oracle
+        self.o = oracle
+        self.wl = wl
+        self.pool = min(pool_rows, wl.M)
+        if wl.kind == "linear":
+            d = workloads.make(wl, rows=slice(0, self.pool))
+            self.x = d["x"]
+            self.wq, self.sw = oracle.quantize_weight(d["w"])
+            self.bias = d["bias"]
+        else:
+            d = workloads.make(wl)
+            self.xq, self.sa = d["xq"][:self.pool], d["scale_a"][:self.pool]
+            self.wq, self.sw, self.bias = d["wq"], d["scale_w"], d["bias"]
+        self.threads = oracle.default_threads()
+
+    def sample(self, rows: int, cols: int, i: int = 0) -> float:
+        r0 = (i * rows) % max(1, self.pool - rows + 1)
+        sl = slice(r0, r0 + rows)
+        wq, sw, bias = self.wq[:cols], self.sw[:cols], self.bias[:cols]
+        t0 = time.perf_counter()
+        if self.wl.kind == "linear":
+            self.o.linear(self.x[sl], wq, sw, bias)
+        else:
+            self.o.epilogue(self.o.gemm_i64(self.xq[sl], wq), self.sa[sl], sw, bias)
+        return time.perf_counter() - t0
+
+
+def size_sample(work: OracleWork, seconds: float) -> tuple[int, int]:
+    """Rows x columns of one oracle sample taking about `seconds`."""
+    wl = work.wl
+    t1 = max(work.sample(1, wl.N), 1e-6)
+    rows = int(seconds / t1)
+    if rows >= 1:
+        return min(rows, work.pool), wl.N
+    cols = max(8, int(wl.N * seconds / t1) // 8 * 8)
+    return 1, min(cols, wl.N)
+
+
+def cpu_baseline(wl: workloads.Workload, budget_s: float = 12.0) -> dict:
+    work = OracleWork(wl)
+    rows, cols = size_sample(work, budget_s)
+    dt = work.sample(rows, cols)
+    ops = 2.0 * rows * cols * wl.K
+    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": work.threads, "kind": "oracle",
+            "sample": f"{rows} of {wl.M} tokens x {cols} of {wl.N} output channels of {wl.name} "
+                      f"(K={wl.K}): whole layer (quantize + exact GEMM + epilogue), {dt:.2f} s",
+            "seconds": dt}
+
+
+def run_reference(args, wl) -> None:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    work = OracleWork(wl)
+    budget = 120.0
+    rows, cols = size_sample(work, budget / max(1, args.steps + args.warmup))
+    for i in range(args.warmup):
+        work.sample(rows, cols, i)
+    total = 0.0
+    for i in range(args.steps):
+        total += work.sample(rows, cols, args.warmup + i)
+    ops = 2.0 * rows * cols * wl.K * args.steps
+    value = ops / total / 1e12
+    sample = (f"{rows} of {wl.M} tokens x {cols} of {wl.N} output channels of {wl.name} per step "
+              f"(K={wl.K}), whole layer")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64",
+            "data": "synthetic", "config": wl_config(wl),
+            "cpu_baseline": {"value": value, "unit": "TOPS", "cores": work.threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def wl_config(wl) -> dict:
+    return {"workload": f"{wl.name}: {wl.note}", "M": wl.M, "N": wl.N, "K": wl.K,
+            "l2": "rotating buffer sets, combined footprint > 3x L2"}
+
+
+# ------------------------------------------------------------- native arm
+
+
+def run_native(args, wl) -> None:
+    import w8a8_int8_gemm_b200 as w8
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # seeded inputs; each rank has its own token batch, the weight is replicated
+    M, N, K = wl.M, wl.N, wl.K
+    if wl.kind != "linear":
+        raise SystemExit(f"workload {wl.name} gives int8 codes; bench the linear-layer workloads")
+    d = workloads.make(wl, rows=slice(rank * M, (rank + 1) * M))
+    w32 = torch.from_numpy(d["w"]).to(dev)
+    x_host = torch.from_numpy(d["x"].view(np.int16)).view(torch.bfloat16)
+    bias = torch.from_numpy(d["bias"].view(np.int16)).view(torch.bfloat16).to(dev)
+    wq0, sw = w8.w8a8_quantize_weight(w32)
+    del w32
+
+    set_bytes = M * K * 2 + N * K + M * K + M * N * 2 + 4 * M
+    nsets = max(2, int(np.ceil(3 * L2_BYTES / set_bytes)))
+    sets = []
+    for i in range(nsets):
+        x = x_host.to(dev) if i == 0 else torch.roll(sets[0]["x"], shifts=i, dims=0)
+        sets.append({"x": x.contiguous(), "wq": wq0 if i == 0 else wq0.clone(),
+                     "xq": torch.empty((M, K), dtype=torch.int8, device=dev),
+                     "sa": torch.empty((M,), dtype=torch.float32, device=dev),
+                     "out": torch.empty((M, N), dtype=torch.bfloat16, device=dev)})
+
+    def step(i, evs=None):
+        s = sets[i % nsets]
+        if evs is not None:
+            evs[0].record(stream)
+        w8.w8a8_quantize_act(s["x"], xq=s["xq"], scale_a=s["sa"], stream=stream)
+        if evs is not None:
+            evs[1].record(stream)
+        w8.w8a8_gemm(s["xq"], s["wq"], s["sa"], sw, bias, out=s["out"], stream=stream)
+        if evs is not None:
+            evs[2].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if w8.w8a8_read_device_error() != 0:
+        raise SystemExit("a kernel wait timed out during warm-up")
+
+    # timed region
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    start.record(stream)
+    for i in range(args.steps):
+        step(i, evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    elapsed_ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    code = w8.w8a8_read_device_error()
+    if code != 0:
+        raise SystemExit(f"a kernel wait timed out in the timed region (site {code})")
+
+    q_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    g_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    ms_step = elapsed_ms / args.steps
+    ops = 2.0 * M * N * K
+    value = ops * world / (ms_step * 1e-3) / 1e12
+
+    peaks = measured_peaks()
+    gemm_ms = statistics.fmean(g_ms)
+    quant_ms = statistics.fmean(q_ms)
+    int8_peak = peaks["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
+    gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
+    quant_bytes = 3 * M * K + 4 * M
+    quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
+    traffic = ncu_traffic(wl.name)
+
+    result = None
+    if rank == 0:
+        e2e = run_e2e(w8, wl, x_host, sets[0]["wq"], sw, bias, dev, stream, args)
+        ctx = context_baselines(wl, d, sets[0], sw, bias, dev, args) if not args.no_context else None
+        cpu = cpu_baseline(wl) if (world == 1 and not args.no_cpu_baseline) else None
+        cfg = wl_config(wl)
+        cfg["parallelism"] = f"dp{world} (independent token batches, replicated weight)"
+        cfg["gemm_config"] = w8.w8a8_select_config(M, N, K)
+        cfg["buffer_sets"] = nsets
+        cfg["footprint_mb"] = round(nsets * set_bytes / 2 ** 20, 1)
+        result = {
+            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded; stands in for Ideogram 4.0 "
+            "DiT activations and weights, which are not available)", "config": cfg,
+            "roofline": {"bound": "tensor", "achieved": gemm_tops, "peak": int8_peak, "unit": "TOPS",
+                         "frac": gemm_tops / int8_peak,
+                         "traffic": traffic["dram_bytes_per_launch"] if traffic else None,
+                         "kernel": "gemm_w8a8_kernel",
+                         "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x "
+                                        f"{NOMINAL_INT8_OVER_BF16} (nominal int8/bf16 ratio)"},
+            "gemm": {"ms": gemm_ms, "tops": gemm_tops, "pct_of_spec_4p5_pops": 100 * gemm_tops / SPEC_INT8_POPS,
+                     "algorithmic_bytes": M * K + N * K + 2 * M * N + 4 * M + 4 * N + 2 * N},
+            "quantizer": {"ms": quant_ms, "gbs": quant_gbs, "frac_of_measured_hbm": quant_gbs / peaks["hbm_gbs"],
+                          "frac_of_8tbs": quant_gbs / 8000.0, "bytes": quant_bytes},
+            "e2e": e2e, "gpu_launches": 2 * args.steps, "clocks": clocks,
+            "cpu_baseline": cpu, "context": ctx,
+        }
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def run_e2e(w8, wl, x_host, wq, sw, bias, dev, stream, args) -> dict:
+    """The public API with host buffers: pinned host X -> device, w8a8_linear,
+    result -> pinned host, every step, timed on the device."""
+    M, N, K = wl.M, wl.N, wl.K
+    xh = x_host.pin_memory()
+    oh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    od = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    sa = torch.empty((M,), dtype=torch.float32, device=dev)
+
+    def one():
+        xd.copy_(xh, non_blocking=True)
+        w8.w8a8_linear(xd, wq, sw, bias, out=od, ws_xq=xq, ws_scale_a=sa, stream=stream)
+        oh.copy_(od, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize(dev)
+    steps = args.e2e_steps
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b) / steps
+    return {"value": 2.0 * M * N * K / (ms * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": ms,
+            "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "steps": steps}
+
+
+def context_baselines(wl, d, s0, sw, bias, dev, args) -> dict:
+    """Context on the same shape: torch bf16 matmul (+bias) and the
+    dequantize-to-bf16-then-bf16-GEMM path the paper replaces."""
+    M, N, K = wl.M, wl.N, wl.K
+    x = s0["x"]
+    w_bf16 = torch.from_numpy(d["w"]).to(dev).to(torch.bfloat16)
+    wq = s0["wq"]
+
+    def bf16_mm():
+        return torch.addmm(bias, x, w_bf16.t())
+
+    def dequant_path():
+        # the production "INT8" forward: quantize, dequantize to bf16, bf16 GEMM
+        xf = x.float()
+        sa = xf.abs().amax(dim=1, keepdim=True) / 127.0
+        xq = torch.clamp(torch.round(xf / torch.where(sa > 0, sa, torch.ones_like(sa))), -127, 127)
+        xd = (xq * sa).to(torch.bfloat16)
+        wd = (wq.float() * sw[:, None]).to(torch.bfloat16)
+        return torch.addmm(bias, xd, wd.t())
+
+    out = {}
+    for name, fn in (("bf16_matmul", bf16_mm), ("dequant_to_bf16_path", dequant_path)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        n = 20
+        a.record()
+        for _ in range(n):
+            fn()
+        b.record()
+        torch.cuda.synchronize(dev)
+        ms = a.elapsed_time(b) / n
+        out[name] = {"ms": ms, "tops": 2.0 * M * N * K / (ms * 1e-3) / 1e12}
+    del w_bf16
+    return out
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=6000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-context", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    wl = workloads.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_native(args, wl)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

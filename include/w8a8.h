@@ -1,0 +1,200 @@
+/*
+ * w8a8.h -- C ABI of the B200 (sm_100a) W8A8 linear layer.
+ *
+ * The operation is the one described in "Realizing Native INT8 Compute for
+ * Diffusion Transformers on Consumer GPUs: A Fused INT8 GEMM Kernel for
+ * Ideogram 4.0" (arXiv 2606.14598), abstract: post-training W8A8
+ * quantization of a diffusion transformer's linear layers, computed as an
+ * int8 x int8 -> int32 GEMM on the tensor cores with the per-token x
+ * per-channel dequantization and the bias folded into the GEMM's epilogue,
+ * in place of a dequantize-to-bf16-then-bf16-GEMM forward.  A linear layer
+ * here is y = x W^T + b (the nn.Linear convention):
+ *
+ *   scale_a[m] = fl32(max_k |x[m,k]| / 127)                       per token
+ *   xq[m,k]    = clamp(rne(fl32(x[m,k] / scale_a[m])), -127, 127)
+ *   acc[m,n]   = sum_k xq[m,k] * wq[n,k]                    exact, int32
+ *   out[m,n]   = bf16_rne((fl32(acc[m,n]) * scale_a[m]) * scale_w[n] + bias[n])
+ *
+ * The abstract gives no formulas; the readings above (symmetric absmax/127
+ * scales, round to nearest even, clamp to +-127, a zero scale giving all-zero
+ * codes, this epilogue order with no fused multiply-add) are the library's
+ * definition.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.   Every array argument is DEVICE memory on the current CUDA device,
+ *           allocated and owned by the caller; the library never allocates
+ *           device memory and never frees caller memory.  (It keeps a small
+ *           host-side cache of device properties.)
+ * Layout.   Row-major.  x: bf16 [M, K]; xq: int8 [M, K]; wq: int8 [N, K]
+ *           (the nn.Linear weight layout, so both GEMM operands are
+ *           K-contiguous); out: bf16 [M, N]; scale_a: fp32 [M]; scale_w:
+ *           fp32 [N]; bias: bf16 [N].  bf16 is passed as void* (raw 16-bit
+ *           IEEE bfloat16 values).
+ * Async.    Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy
+ *           default stream) and the call returns without synchronizing.
+ *           Errors found before the launch are returned; a wait inside a
+ *           kernel that runs out of time (see w8a8_read_device_error) is
+ *           reported later.
+ * Shapes.   M >= 0 and N >= 0 (M == 0 or N == 0 is a valid empty call that
+ *           launches nothing and returns W8A8_OK); 16 <= K <= 133144 and
+ *           K % 16 == 0 (16-byte rows for the tensor-memory-access engine;
+ *           K * 127^2 < 2^31 keeps the int32 accumulator exact);
+ *           N % 8 == 0 (16-byte output rows); M, N < 2^31.
+ * Alignment. Every pointer is 16-byte aligned; otherwise W8A8_ERR_ALIGNMENT.
+ * Device.   Compute capability 10.0 (B200, sm_100a); otherwise
+ *           W8A8_ERR_UNSUPPORTED_DEVICE.
+ * Errors.   Argument errors are detected before any device work and launch
+ *           nothing.  A CUDA launch error is returned as W8A8_ERR_LAUNCH.
+ */
+#ifndef W8A8_H
+#define W8A8_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define W8A8_API __attribute__((visibility("default")))
+#else
+#define W8A8_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st* w8a8_stream_t;
+
+typedef enum {
+    W8A8_OK = 0,
+    W8A8_ERR_INVALID_ARG = 1,         /* bad shape, stride, or NULL pointer */
+    W8A8_ERR_ALIGNMENT = 2,           /* a pointer or row stride is not 16-byte aligned */
+    W8A8_ERR_UNSUPPORTED_DEVICE = 3,  /* current device is not sm_100 */
+    W8A8_ERR_LAUNCH = 4,              /* CUDA refused the launch */
+    W8A8_ERR_TIMEOUT = 5,             /* a kernel's bounded wait ran out (see w8a8_read_device_error) */
+    W8A8_ERR_CUDA = 6                 /* another CUDA runtime error */
+} w8a8_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+W8A8_API const char* w8a8_status_string(int status);
+
+/* ABI version of this header: 100 * major + minor. */
+W8A8_API int w8a8_abi_version(void);
+
+/*
+ * Per-token activation quantization (the paper's per-token activation
+ * quantizer; abstract: "per-token" dequantization of the W8A8 GEMM).
+ *   x       bf16 [M, K], row stride ldx elements (ldx >= K, ldx % 8 == 0)
+ *   xq      int8 [M, K] out, row stride ldxq bytes (ldxq >= K, ldxq % 16 == 0)
+ *   scale_a fp32 [M] out
+ * One warp per token row, 16-byte loads, a shuffle max-reduction, packed
+ * int8 stores.  Results are bit-exact to the definition in the header.
+ */
+W8A8_API w8a8_status w8a8_quantize_act(const void* x, int64_t M, int64_t K, int64_t ldx,
+                              int8_t* xq, int64_t ldxq, float* scale_a, w8a8_stream_t stream);
+
+/*
+ * Per-output-channel weight quantization (abstract: post-training W8A8
+ * quantization, dequantized per channel in the epilogue).  Same rule as the
+ * activation quantizer applied to each row of an fp32 weight:
+ *   w       fp32 [N, K], row stride ldw elements (ldw >= K, ldw % 4 == 0)
+ *   wq      int8 [N, K] out, row stride ldwq bytes (ldwq >= K, ldwq % 16 == 0)
+ *   scale_w fp32 [N] out
+ * Used once per weight at load time, not per forward.
+ */
+W8A8_API w8a8_status w8a8_quantize_weight(const float* w, int64_t N, int64_t K, int64_t ldw,
+                                 int8_t* wq, int64_t ldwq, float* scale_w, w8a8_stream_t stream);
+
+/*
+ * Fused W8A8 GEMM (abstract: "int8xint8->int32 ... with per-token x
+ * per-channel dequantization and bias folded into the epilogue"):
+ *   out[m,n] = bf16_rne((fl32(sum_k xq[m,k]*wq[n,k]) * scale_a[m]) * scale_w[n] + bias[n])
+ *   xq [M, K] int8, wq [N, K] int8 (row strides K), scale_a [M], scale_w [N]
+ *   fp32, bias [N] bf16 or NULL (zero bias), out [M, N] bf16 (row stride N).
+ * tcgen05 int8 tensor-core kernel with int32 accumulators in tensor memory;
+ * the tile configuration is chosen per shape (w8a8_select_config).
+ */
+W8A8_API w8a8_status w8a8_gemm(const int8_t* xq, const int8_t* wq, const float* scale_a,
+                      const float* scale_w, const void* bias, void* out,
+                      int64_t M, int64_t N, int64_t K, w8a8_stream_t stream);
+
+/*
+ * The whole W8A8 linear layer (abstract: the fused kernel "dropped into the
+ * ... linear layers in place of the dequantize-to-bf16 path"):
+ * w8a8_quantize_act of x into the caller's workspace, then w8a8_gemm.
+ *   x [M, K] bf16 (row stride K); wq, scale_w, bias, out as in w8a8_gemm;
+ *   ws_xq int8 [M, K] and ws_scale_a fp32 [M]: caller-owned workspace that
+ *   receives the quantized activations and their scales (readable after the
+ *   call completes).
+ */
+W8A8_API w8a8_status w8a8_linear(const void* x, const int8_t* wq, const float* scale_w, const void* bias,
+                        void* out, int8_t* ws_xq, float* ws_scale_a,
+                        int64_t M, int64_t N, int64_t K, w8a8_stream_t stream);
+
+/*
+ * The GEMM without the epilogue: raw int32 accumulators
+ *   acc[m,n] = sum_k xq[m,k]*wq[n,k], acc int32 [M, N] (row stride N).
+ * The abstract states the int32 accumulation is bit-exact against a library
+ * integer matmul; this entry point exposes it for that check.
+ */
+W8A8_API w8a8_status w8a8_gemm_i32(const int8_t* xq, const int8_t* wq, int32_t* acc,
+                          int64_t M, int64_t N, int64_t K, w8a8_stream_t stream);
+
+/*
+ * Per-shape GEMM configuration (abstract: the kernel is "autotuned per GEMM
+ * shape"; here a static cost model over a measured table of tile shapes).
+ */
+typedef struct {
+    int32_t block_m;       /* rows of the output tile per CTA: 128 */
+    int32_t block_n;       /* columns of the output tile: 128 or 256 */
+    int32_t stages;        /* depth of the shared-memory operand ring */
+    int32_t grid;          /* persistent CTAs launched (<= number of SMs) */
+    int32_t raster_group;  /* M tiles walked together before moving along N */
+    int32_t reserved[3];   /* zero */
+} w8a8_gemm_config;
+
+/* The configuration w8a8_gemm would use for this shape on the current
+ * device.  Shapes are validated as for w8a8_gemm. */
+W8A8_API w8a8_status w8a8_select_config(int64_t M, int64_t N, int64_t K, w8a8_gemm_config* cfg);
+
+/* w8a8_gemm / w8a8_gemm_i32 with an explicit configuration (cfg NULL means
+ * the selected one).  block_m must be 128, block_n 128 or 256, stages within
+ * what shared memory holds (2..4 at block_n 256, 2..6 at 128), 1 <= grid,
+ * 1 <= raster_group; anything else is W8A8_ERR_INVALID_ARG.  For sweeps and
+ * tests: every valid configuration computes the same result. */
+W8A8_API w8a8_status w8a8_gemm_ex(const int8_t* xq, const int8_t* wq, const float* scale_a,
+                         const float* scale_w, const void* bias, void* out,
+                         int64_t M, int64_t N, int64_t K, const w8a8_gemm_config* cfg,
+                         w8a8_stream_t stream);
+W8A8_API w8a8_status w8a8_gemm_i32_ex(const int8_t* xq, const int8_t* wq, int32_t* acc,
+                             int64_t M, int64_t N, int64_t K, const w8a8_gemm_config* cfg,
+                             w8a8_stream_t stream);
+
+/*
+ * Every wait inside the library's kernels is bounded in time.  When one
+ * runs out the kernel records a nonzero code in a device-side error word,
+ * finishes its own in-flight copies, frees its tensor memory and exits, so
+ * the CUDA context stays usable and the output is incomplete.
+ * w8a8_read_device_error synchronizes the current device, stores the word
+ * in *code (0 = no timeout since the last clear), clears it if `clear` is
+ * nonzero, and returns W8A8_ERR_TIMEOUT if the word was nonzero.
+ */
+W8A8_API w8a8_status w8a8_read_device_error(int32_t* code, int32_t clear);
+
+/* Time limit of every bounded wait, in nanoseconds (default 2e9; values
+ * below 1e5 are raised to 1e5).  Applies to launches made after the call. */
+W8A8_API w8a8_status w8a8_set_wait_timeout_ns(int64_t ns);
+
+/*
+ * Self-test of the timeout path: launches one small kernel that waits on a
+ * barrier nothing ever completes, with the given limit (>= 1e5 ns), so that
+ * the wait runs out by construction and the error word is set.  No other
+ * state is touched.  Used to check failure detection without any fault.
+ */
+W8A8_API w8a8_status w8a8_selftest_wait_timeout(int64_t timeout_ns, w8a8_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W8A8_H */

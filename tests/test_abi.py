@@ -1,0 +1,78 @@
+"""The C ABI on the host (no GPU needed): the shared object loads, exports
+every function include/w8a8.h declares and nothing else, and rejects bad
+arguments before touching any device."""
+import ctypes
+import subprocess
+
+import pytest
+
+import __graft_entry__
+
+
+@pytest.fixture(scope="module")
+def w8():
+    __graft_entry__.build()
+    import w8a8_int8_gemm_b200 as mod
+    return mod
+
+
+def test_exports_match_header(w8):
+    declared = set(w8.exported_names())
+    assert {"w8a8_quantize_act", "w8a8_gemm", "w8a8_linear", "w8a8_gemm_i32"} <= declared
+    lib = w8.raw_lib()
+    for name in declared:
+        assert hasattr(lib, name), f"{name} declared but not exported"
+    out = subprocess.run(["nm", "-D", "--defined-only", w8.lib_path], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    ours = {n for n in exported if n.startswith("w8a8_")}
+    assert ours == declared, f"exported {sorted(ours ^ declared)} differ from the header"
+
+
+def test_status_strings(w8):
+    assert w8.w8a8_status_string(0) == "ok"
+    for s in range(1, 7):
+        assert w8.w8a8_status_string(s) not in ("ok", "unknown status")
+    assert w8.w8a8_status_string(99) == "unknown status"
+    assert w8.w8a8_abi_version() == 100
+
+
+def _gemm_i32(lib, xq, wq, acc, M, N, K):
+    return lib.w8a8_gemm_i32(xq, wq, acc, M, N, K, None)
+
+
+def test_host_validation_without_device(w8):
+    lib = w8.raw_lib()
+    A = 0x10000  # fake 16-byte-aligned addresses: never dereferenced on these paths
+    # shapes
+    assert _gemm_i32(lib, A, A, A, 4, 8, 24) == 1          # K % 16
+    assert _gemm_i32(lib, A, A, A, 4, 8, 0) == 1           # K == 0
+    assert _gemm_i32(lib, A, A, A, 4, 12, 32) == 1         # N % 8
+    assert _gemm_i32(lib, A, A, A, -1, 8, 32) == 1         # negative M
+    assert _gemm_i32(lib, A, A, A, 4, 8, 133152) == 1      # K * 127^2 >= 2^31
+    # empty problems succeed without launching
+    assert _gemm_i32(lib, A, A, A, 0, 8, 32) == 0
+    assert _gemm_i32(lib, A, A, A, 4, 0, 32) == 0
+    # null and misaligned pointers
+    assert _gemm_i32(lib, None, A, A, 4, 8, 32) == 1
+    assert _gemm_i32(lib, A + 8, A, A, 4, 8, 32) == 2
+    assert _gemm_i32(lib, A, A, A + 4, 4, 8, 32) == 2
+    assert lib.w8a8_gemm(A, A, A, A, A + 2, A, 4, 8, 32, None) == 2   # misaligned bias
+    assert lib.w8a8_gemm(A, A, None, A, None, A, 4, 8, 32, None) == 1  # missing scale_a
+    # quantizers
+    assert lib.w8a8_quantize_act(A, 4, 32, 16, A, 32, A, None) == 1    # ldx < K
+    assert lib.w8a8_quantize_act(A, 4, 32, 36, A, 32, A, None) == 2    # ldx * 2 not 16-byte
+    assert lib.w8a8_quantize_act(A, 4, 32, 32, A, 40, A, None) == 2    # ldxq not 16-byte
+    assert lib.w8a8_quantize_act(A, 0, 32, 32, A, 32, A, None) == 0
+    assert lib.w8a8_quantize_weight(A, 4, 32, 34, A, 32, A, None) == 2  # ldw * 4 not 16-byte
+    # linear validates the whole call first
+    assert lib.w8a8_linear(A, A, A, None, A, A, A, 4, 12, 32, None) == 1
+    assert lib.w8a8_linear(A, A, A, None, A, A + 1, A, 4, 8, 32, None) == 2
+    assert lib.w8a8_linear(A, A, A, None, A, A, A, 0, 8, 32, None) == 0
+    # explicit configurations
+    cfg = w8.GemmConfig(block_m=128, block_n=200, stages=4, grid=1, raster_group=1)
+    assert lib.w8a8_gemm_i32_ex(A, A, A, 4, 8, 32, ctypes.byref(cfg), None) == 1
+    cfg = w8.GemmConfig(block_m=128, block_n=256, stages=5, grid=1, raster_group=1)
+    assert lib.w8a8_gemm_i32_ex(A, A, A, 4, 8, 32, ctypes.byref(cfg), None) == 1
+    assert lib.w8a8_select_config(4, 8, 32, None) == 1
+    assert lib.w8a8_selftest_wait_timeout(10, None) == 1

@@ -1,0 +1,113 @@
+"""GPU parity of the whole W8A8 linear layer (w8a8_linear) against the CPU
+oracle, on every DiT workload at full size in the launch configuration the
+benchmark uses (the selected tile configuration, all tokens in one call):
+
+* the weight is quantized on both sides from the same seeded fp32 weight
+  (codes and scales must agree bit for bit first);
+* per-token codes and scales of every row are bit-exact;
+* the bf16 output is within 1 ulp of the oracle on sampled rows (first,
+  last, tile-boundary and random rows) -- the oracle's exact GEMM on every
+  row of the large shapes would take minutes of CPU -- and has no NaN;
+* the cosine similarity with the unquantized fp64 product is reported and
+  must be high (the paper reports cosine 1.0 for its kernel).
+
+Paper: "Realizing Native INT8 Compute for Diffusion Transformers on Consumer
+GPUs" (arXiv 2606.14598), abstract."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.util import bf16_bits_to_torch, bf16_ulp_diff, is_nan_bits, sample_rows, torch_bf16_to_bits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def w8():
+    import w8a8_int8_gemm_b200 as mod
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return mod
+
+
+def _run(w8, name, n_sample):
+    wl = workloads.WORKLOADS[name]
+    d = workloads.make(wl)
+    dev = torch.device("cuda")
+    wq, sw = w8.w8a8_quantize_weight(torch.from_numpy(d["w"]).to(dev))
+    x = bf16_bits_to_torch(d["x"], dev)
+    bias = bf16_bits_to_torch(d["bias"], dev)
+    xq = torch.empty((wl.M, wl.K), dtype=torch.int8, device=dev)
+    sa = torch.empty((wl.M,), dtype=torch.float32, device=dev)
+    out = w8.w8a8_linear(x, wq, sw, bias, ws_xq=xq, ws_scale_a=sa)
+    torch.cuda.synchronize()
+    assert w8.w8a8_read_device_error() == 0
+
+    wq_o, sw_o = oracle.quantize_weight(d["w"])
+    assert np.array_equal(sw.cpu().numpy().view(np.uint32), sw_o.view(np.uint32)), "weight scales differ"
+    assert np.array_equal(wq.cpu().numpy(), wq_o), "weight codes differ"
+
+    xq_o, sa_o = oracle.quantize_act(d["x"])
+    assert np.array_equal(sa.cpu().numpy().view(np.uint32), sa_o.view(np.uint32)), "token scales differ"
+    assert np.array_equal(xq.cpu().numpy(), xq_o), "token codes differ"
+
+    got = torch_bf16_to_bits(out)
+    assert not is_nan_bits(got).any(), "NaN in the output"
+    rows = np.arange(wl.M) if n_sample is None else sample_rows(wl.M, n_sample, wl.seed)
+    out_o, xq_r, sa_r, acc_o = oracle.linear(d["x"][rows], wq_o, sw_o, d["bias"])
+    ulp = bf16_ulp_diff(got[rows], out_o)
+    assert ulp.max() <= 1, f"max {ulp.max()} ulp at {np.argwhere(ulp > 1)[:3].tolist()}"
+
+    # the paper's accuracy metric, against the unquantized product
+    xf = oracle.bf16_bits_to_f32(d["x"][rows[:8]]).astype(np.float64)
+    ref = xf @ d["w"].astype(np.float64).T + oracle.bf16_bits_to_f32(d["bias"]).astype(np.float64)
+    y = torch.from_numpy(got[rows[:8]].view(np.int16)).view(torch.bfloat16).double().numpy()
+    cos = float((ref * y).sum() / np.sqrt((ref * ref).sum() * (y * y).sum()))
+    assert cos > 0.999, cos
+    return ulp
+
+
+def test_linear_tiny_all_rows(w8):
+    ulp = _run(w8, "tiny", None)
+    assert ulp.max() <= 1
+
+
+@pytest.mark.parametrize("name", ["qkv_768", "mlp_up_1024"])
+def test_linear_dit_workloads(w8, name):
+    _run(w8, name, 40)
+
+
+@pytest.mark.parametrize("name", ["sweep_qkv", "sweep_out", "sweep_up", "sweep_down"])
+def test_linear_block_sweep(w8, name):
+    _run(w8, name, 24)
+
+
+def test_linear_ragged(w8):
+    """Token counts that are not multiples of the tile, N not a multiple of 256."""
+    rng = np.random.default_rng(5)
+    dev = torch.device("cuda")
+    for M, N, K in [(1, 8, 16), (77, 136, 144), (130, 392, 1040)]:
+        x_bits = workloads._to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+        w = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+        bias_bits = workloads.gen_bias(N, M)
+        wq, sw = w8.w8a8_quantize_weight(torch.from_numpy(w).to(dev))
+        out = w8.w8a8_linear(bf16_bits_to_torch(x_bits, dev), wq, sw, bf16_bits_to_torch(bias_bits, dev))
+        torch.cuda.synchronize()
+        wq_o, sw_o = oracle.quantize_weight(w)
+        out_o, *_ = oracle.linear(x_bits, wq_o, sw_o, bias_bits)
+        assert bf16_ulp_diff(torch_bf16_to_bits(out), out_o).max() <= 1, (M, N, K)
+
+
+def test_linear_zero_tokens_give_bias(w8):
+    dev = torch.device("cuda")
+    M, N, K = 40, 264, 96
+    x = torch.zeros((M, K), dtype=torch.bfloat16, device=dev)
+    x[3, 5] = 2.0
+    wq = torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev)
+    sw = torch.rand(N, device=dev) * 0.01
+    bias = (torch.randn(N, device=dev) * 0.1).to(torch.bfloat16)
+    out = w8.w8a8_linear(x, wq, sw, bias)
+    torch.cuda.synchronize()
+    rows = [r for r in range(M) if r != 3]
+    assert torch.equal(out[rows], bias.expand(M - 1, N))

@@ -1,0 +1,130 @@
+"""GPU parity of the row quantizers (w8a8_quantize_act, w8a8_quantize_weight)
+against the CPU oracle: int8 codes and fp32 scales must be bit-exact.
+
+Paper: "Realizing Native INT8 Compute for Diffusion Transformers on Consumer
+GPUs" (arXiv 2606.14598), abstract -- per-token activation quantization and
+per-channel weight quantization of W8A8."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests import oracle_pins as P
+from tests.util import bf16_bits_to_torch
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def w8():
+    import w8a8_int8_gemm_b200 as mod
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return mod
+
+
+def _run_act(w8, bits, ldx_pad=0, ldq_pad=0):
+    M, K = bits.shape
+    dev = torch.device("cuda")
+    xfull = torch.zeros((M, K + ldx_pad), dtype=torch.bfloat16, device=dev)
+    xfull[:, :K] = bf16_bits_to_torch(bits, dev)
+    x = xfull[:, :K]
+    qfull = torch.full((M, K + ldq_pad), 99, dtype=torch.int8, device=dev)
+    q = qfull[:, :K]
+    q, s = w8.w8a8_quantize_act(x, xq=q)
+    torch.cuda.synchronize()
+    if ldq_pad:
+        assert (qfull[:, K:] == 99).all(), "quantizer wrote past K in the padded output rows"
+    return q.cpu().numpy(), s.cpu().numpy()
+
+
+def _assert_same(q, s, bits):
+    qo, so = oracle.quantize_act(bits)
+    assert np.array_equal(s.view(np.uint32), so.view(np.uint32)), "scale_a differs from the oracle"
+    bad = np.argwhere(q != qo)
+    assert bad.size == 0, f"{len(bad)} codes differ, first at {bad[:3].tolist()}"
+
+
+@pytest.mark.parametrize("M,K", [(1, 16), (7, 48), (9, 272), (63, 1024), (64, 2048), (33, 3072),
+                                 (17, 4096), (5, 4112), (3, 12288), (2, 20000 // 16 * 16)])
+def test_act_random_shapes(w8, M, K):
+    rng = np.random.default_rng(M * 100003 + K)
+    x = rng.standard_normal((M, K)).astype(np.float32) * np.float32(3.0)
+    bits = P.to_bits(x)
+    q, s = _run_act(w8, bits)
+    _assert_same(q, s, bits)
+
+
+def test_act_edge_rows(w8):
+    """Zero rows, -0, a single non-zero, bf16 subnormals, exact ties, huge values."""
+    rng = np.random.default_rng(3)
+    K = 512
+    x = P.edge_rows(K, rng)
+    bits = P.to_bits(x)
+    # rows from the hand-worked fixture, padded with zeros to K
+    for xs, _, _ in P.read_rows("quant_act_rows.txt"):
+        r = np.zeros(K, np.float32)
+        vals = np.array([float(v) for v in xs], np.float32)
+        r[:len(vals)] = vals
+        bits = np.concatenate([bits, P.bf16_bits(r)[None, :]])
+    q, s = _run_act(w8, bits)
+    _assert_same(q, s, bits)
+
+
+def test_act_strided(w8):
+    rng = np.random.default_rng(4)
+    bits = P.to_bits(rng.standard_normal((37, 320)).astype(np.float32))
+    q, s = _run_act(w8, bits, ldx_pad=24, ldq_pad=48)
+    _assert_same(q, s, bits)
+
+
+@pytest.mark.parametrize("name", ["tiny", "qkv_768", "mlp_up_1024"])
+def test_act_workloads_full(w8, name):
+    """Every row of the workload's activations, bit-exact."""
+    wl = workloads.WORKLOADS[name]
+    bits = workloads.gen_activations(wl.M, wl.K, wl.seed, wl.outliers)
+    q, s = _run_act(w8, bits)
+    _assert_same(q, s, bits)
+
+
+def test_act_long_k_workload_full(w8):
+    """The 9216 x 12288 input of the MLP down-projection sweep (second-pass path)."""
+    wl = workloads.WORKLOADS["sweep_down"]
+    bits = workloads.gen_activations(wl.M, wl.K, wl.seed, wl.outliers)
+    q, s = _run_act(w8, bits)
+    _assert_same(q, s, bits)
+
+
+def test_act_empty(w8):
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    q, s = w8.w8a8_quantize_act(x)
+    assert q.shape == (0, 64) and s.shape == (0,)
+
+
+@pytest.mark.parametrize("N,K", [(128, 256), (136, 48), (12288, 3072), (3072, 12288)])
+def test_weight_quant(w8, N, K):
+    rng = np.random.default_rng(N + K)
+    w = rng.standard_normal((N, K)).astype(np.float32) * np.float32(0.02)
+    wq, sw = w8.w8a8_quantize_weight(torch.from_numpy(w).cuda())
+    torch.cuda.synchronize()
+    wq_o, sw_o = oracle.quantize_weight(w)
+    assert np.array_equal(sw.cpu().numpy().view(np.uint32), sw_o.view(np.uint32))
+    assert np.array_equal(wq.cpu().numpy(), wq_o)
+
+
+def test_weight_quant_golden_and_subnormal(w8):
+    """Hand-worked weight rows, including an fp32 subnormal row that clamps
+    and one whose scale underflows to zero."""
+    K = 64
+    rows = []
+    for ws, _, _ in P.read_rows("quant_weight_rows.txt"):
+        r = np.zeros(K, np.float32)
+        vals = np.array([P.parse_num(v) for v in ws], np.float32)
+        r[:len(vals)] = vals
+        rows.append(r)
+    w = np.stack(rows)
+    wq, sw = w8.w8a8_quantize_weight(torch.from_numpy(w).cuda())
+    torch.cuda.synchronize()
+    wq_o, sw_o = oracle.quantize_weight(w)
+    assert np.array_equal(sw.cpu().numpy().view(np.uint32), sw_o.view(np.uint32))
+    assert np.array_equal(wq.cpu().numpy(), wq_o)

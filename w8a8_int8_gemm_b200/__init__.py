@@ -1,0 +1,317 @@
+"""B200-native W8A8 linear layer: Python binding of libw8a8.so.
+
+The functions below have the names of the C entry points in
+``include/w8a8.h`` and do argument marshalling only: they check that the
+torch tensors have the layout the C ABI expects, allocate outputs the
+caller did not pass (torch is used for device memory and streams), and call
+the library on the current CUDA stream.  Every step of the computation runs
+in the library's CUDA kernels; there is no fallback.  If the shared object
+has not been built, importing this package raises ImportError.
+
+Method: "Realizing Native INT8 Compute for Diffusion Transformers on
+Consumer GPUs: A Fused INT8 GEMM Kernel for Ideogram 4.0" (arXiv
+2606.14598), abstract -- per-token activation quantization, an int8 x int8
+-> int32 GEMM against per-channel int8 weights, and the per-token x
+per-channel dequantization plus bias folded into the GEMM epilogue, bf16 out.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+__all__ = [
+    "W8A8Error", "lib_path", "header_path", "exported_names",
+    "w8a8_status_string", "w8a8_abi_version",
+    "w8a8_quantize_act", "w8a8_quantize_weight", "w8a8_gemm", "w8a8_gemm_ex",
+    "w8a8_gemm_i32", "w8a8_gemm_i32_ex", "w8a8_linear", "w8a8_select_config",
+    "w8a8_read_device_error", "w8a8_set_wait_timeout_ns", "w8a8_selftest_wait_timeout",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_PKG, "libw8a8.so")
+header_path = os.path.join(os.path.dirname(_PKG), "include", "w8a8.h")
+
+W8A8_OK = 0
+W8A8_ERR_TIMEOUT = 5
+
+
+class W8A8Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {w8a8_status_string(status)} (status {status})")
+
+
+class GemmConfig(ctypes.Structure):
+    _fields_ = [("block_m", ctypes.c_int32), ("block_n", ctypes.c_int32), ("stages", ctypes.c_int32),
+                ("grid", ctypes.c_int32), ("raster_group", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
+
+    def as_dict(self) -> dict:
+        return {"block_m": self.block_m, "block_n": self.block_n, "stages": self.stages,
+                "grid": self.grid, "raster_group": self.raster_group}
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(lib_path):
+        raise ImportError(
+            f"{lib_path} is missing: build the CUDA library first "
+            "(python w8a8_int8_gemm_b200/build.py, or __graft_entry__.build())")
+    lib = ctypes.CDLL(lib_path)
+    p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    sigs = {
+        "w8a8_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "w8a8_abi_version": ([], ctypes.c_int),
+        "w8a8_quantize_act": ([p, i64, i64, i64, p, i64, p, p], ctypes.c_int),
+        "w8a8_quantize_weight": ([p, i64, i64, i64, p, i64, p, p], ctypes.c_int),
+        "w8a8_gemm": ([p, p, p, p, p, p, i64, i64, i64, p], ctypes.c_int),
+        "w8a8_gemm_ex": ([p, p, p, p, p, p, i64, i64, i64, ctypes.POINTER(GemmConfig), p], ctypes.c_int),
+        "w8a8_gemm_i32": ([p, p, p, i64, i64, i64, p], ctypes.c_int),
+        "w8a8_gemm_i32_ex": ([p, p, p, i64, i64, i64, ctypes.POINTER(GemmConfig), p], ctypes.c_int),
+        "w8a8_linear": ([p, p, p, p, p, p, p, i64, i64, i64, p], ctypes.c_int),
+        "w8a8_select_config": ([i64, i64, i64, ctypes.POINTER(GemmConfig)], ctypes.c_int),
+        "w8a8_read_device_error": ([ctypes.POINTER(i32), i32], ctypes.c_int),
+        "w8a8_set_wait_timeout_ns": ([i64], ctypes.c_int),
+        "w8a8_selftest_wait_timeout": ([i64, p], ctypes.c_int),
+    }
+    for name, (args, res) in sigs.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+_lib = _load()
+
+
+def exported_names() -> list[str]:
+    """Names of the functions include/w8a8.h declares."""
+    with open(header_path) as fh:
+        text = fh.read()
+    return sorted(set(re.findall(r"W8A8_API\s+[\w\s\*]+?\b(w8a8_\w+)\s*\(", text)))
+
+
+# ------------------------------------------------------------ helpers
+
+
+def _check(status: int, what: str) -> None:
+    if status != W8A8_OK:
+        raise W8A8Error(status, what)
+
+
+def _stream(stream, device) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got {t.dim()}")
+    if t.numel() > 0 and t.stride(-1) != 1:
+        raise ValueError(f"{name} must be contiguous in its last dimension")
+
+
+def _need_contig(t: torch.Tensor, name: str, dtype: torch.dtype, shape: tuple) -> None:
+    _need(t, name, dtype, len(shape))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _cfg(config) -> GemmConfig | None:
+    if config is None:
+        return None
+    if isinstance(config, GemmConfig):
+        return config
+    c = GemmConfig()
+    for k in ("block_m", "block_n", "stages", "grid", "raster_group"):
+        setattr(c, k, int(config[k]))
+    return c
+
+
+# --------------------------------------------------------- entry points
+
+
+def w8a8_status_string(status: int) -> str:
+    return _lib.w8a8_status_string(int(status)).decode()
+
+
+def w8a8_abi_version() -> int:
+    return int(_lib.w8a8_abi_version())
+
+
+def w8a8_quantize_act(x: torch.Tensor, xq: torch.Tensor | None = None, scale_a: torch.Tensor | None = None,
+                      stream=None):
+    """Per-token int8 quantization of bf16 x [M, K] -> (xq int8 [M, K], scale_a fp32 [M])."""
+    _need(x, "x", torch.bfloat16, 2)
+    M, K = x.shape
+    if xq is None:
+        xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if scale_a is None:
+        scale_a = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _need(xq, "xq", torch.int8, 2)
+    if tuple(xq.shape) != (M, K):
+        raise ValueError("xq must have the shape of x")
+    _need_contig(scale_a, "scale_a", torch.float32, (M,))
+    _check(_lib.w8a8_quantize_act(_ptr(x), M, K, x.stride(0) if M else K, _ptr(xq),
+                                  xq.stride(0) if M else K, _ptr(scale_a), _stream(stream, x.device)),
+           "w8a8_quantize_act")
+    return xq, scale_a
+
+
+def w8a8_quantize_weight(w: torch.Tensor, wq: torch.Tensor | None = None, scale_w: torch.Tensor | None = None,
+                         stream=None):
+    """Per-output-channel int8 quantization of fp32 w [N, K] -> (wq int8 [N, K], scale_w fp32 [N])."""
+    _need(w, "w", torch.float32, 2)
+    N, K = w.shape
+    if wq is None:
+        wq = torch.empty((N, K), dtype=torch.int8, device=w.device)
+    if scale_w is None:
+        scale_w = torch.empty((N,), dtype=torch.float32, device=w.device)
+    _need(wq, "wq", torch.int8, 2)
+    if tuple(wq.shape) != (N, K):
+        raise ValueError("wq must have the shape of w")
+    _need_contig(scale_w, "scale_w", torch.float32, (N,))
+    _check(_lib.w8a8_quantize_weight(_ptr(w), N, K, w.stride(0) if N else K, _ptr(wq),
+                                     wq.stride(0) if N else K, _ptr(scale_w), _stream(stream, w.device)),
+           "w8a8_quantize_weight")
+    return wq, scale_w
+
+
+def _gemm_operands(xq, wq):
+    _need(xq, "xq", torch.int8, 2)
+    _need(wq, "wq", torch.int8, 2)
+    M, K = xq.shape
+    N, K2 = wq.shape
+    if K != K2:
+        raise ValueError(f"inner dimensions differ: xq has K={K}, wq has K={K2}")
+    _need_contig(xq, "xq", torch.int8, (M, K))
+    _need_contig(wq, "wq", torch.int8, (N, K))
+    return M, N, K
+
+
+def w8a8_gemm_ex(xq, wq, scale_a, scale_w, bias=None, out=None, config=None, stream=None):
+    """Fused GEMM with an explicit tile configuration (None = selected per shape)."""
+    M, N, K = _gemm_operands(xq, wq)
+    _need_contig(scale_a, "scale_a", torch.float32, (M,))
+    _need_contig(scale_w, "scale_w", torch.float32, (N,))
+    if bias is not None:
+        _need_contig(bias, "bias", torch.bfloat16, (N,))
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    _need_contig(out, "out", torch.bfloat16, (M, N))
+    c = _cfg(config)
+    st = _lib.w8a8_gemm_ex(_ptr(xq), _ptr(wq), _ptr(scale_a), _ptr(scale_w), _ptr(bias), _ptr(out), M, N, K,
+                           ctypes.byref(c) if c is not None else None, _stream(stream, xq.device))
+    _check(st, "w8a8_gemm_ex")
+    return out
+
+
+def w8a8_gemm(xq, wq, scale_a, scale_w, bias=None, out=None, stream=None):
+    """out bf16 [M, N] = bf16((fl32(xq @ wq^T) * scale_a[:, None]) * scale_w[None, :] + bias)."""
+    M, N, K = _gemm_operands(xq, wq)
+    _need_contig(scale_a, "scale_a", torch.float32, (M,))
+    _need_contig(scale_w, "scale_w", torch.float32, (N,))
+    if bias is not None:
+        _need_contig(bias, "bias", torch.bfloat16, (N,))
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    _need_contig(out, "out", torch.bfloat16, (M, N))
+    _check(_lib.w8a8_gemm(_ptr(xq), _ptr(wq), _ptr(scale_a), _ptr(scale_w), _ptr(bias), _ptr(out), M, N, K,
+                          _stream(stream, xq.device)), "w8a8_gemm")
+    return out
+
+
+def w8a8_gemm_i32(xq, wq, acc=None, stream=None, config=None):
+    """Raw int32 accumulators acc [M, N] = xq @ wq^T (exact)."""
+    M, N, K = _gemm_operands(xq, wq)
+    if acc is None:
+        acc = torch.empty((M, N), dtype=torch.int32, device=xq.device)
+    _need_contig(acc, "acc", torch.int32, (M, N))
+    if config is None:
+        st = _lib.w8a8_gemm_i32(_ptr(xq), _ptr(wq), _ptr(acc), M, N, K, _stream(stream, xq.device))
+    else:
+        c = _cfg(config)
+        st = _lib.w8a8_gemm_i32_ex(_ptr(xq), _ptr(wq), _ptr(acc), M, N, K, ctypes.byref(c),
+                                   _stream(stream, xq.device))
+    _check(st, "w8a8_gemm_i32")
+    return acc
+
+
+def w8a8_gemm_i32_ex(xq, wq, acc=None, config=None, stream=None):
+    return w8a8_gemm_i32(xq, wq, acc=acc, stream=stream, config=config)
+
+
+def w8a8_linear(x, wq, scale_w, bias=None, out=None, ws_xq=None, ws_scale_a=None, stream=None):
+    """The W8A8 linear layer: out bf16 [M, N] from bf16 x [M, K] and int8 wq [N, K].
+
+    ws_xq int8 [M, K] and ws_scale_a fp32 [M] receive the quantized
+    activations (allocated here if not given)."""
+    _need(x, "x", torch.bfloat16, 2)
+    M, K = x.shape
+    _need(wq, "wq", torch.int8, 2)
+    N = wq.shape[0]
+    if wq.shape[1] != K:
+        raise ValueError(f"inner dimensions differ: x has K={K}, wq has K={wq.shape[1]}")
+    _need_contig(x, "x", torch.bfloat16, (M, K))
+    _need_contig(wq, "wq", torch.int8, (N, K))
+    _need_contig(scale_w, "scale_w", torch.float32, (N,))
+    if bias is not None:
+        _need_contig(bias, "bias", torch.bfloat16, (N,))
+    dev = x.device
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    if ws_xq is None:
+        ws_xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    if ws_scale_a is None:
+        ws_scale_a = torch.empty((M,), dtype=torch.float32, device=dev)
+    _need_contig(out, "out", torch.bfloat16, (M, N))
+    _need_contig(ws_xq, "ws_xq", torch.int8, (M, K))
+    _need_contig(ws_scale_a, "ws_scale_a", torch.float32, (M,))
+    _check(_lib.w8a8_linear(_ptr(x), _ptr(wq), _ptr(scale_w), _ptr(bias), _ptr(out), _ptr(ws_xq),
+                            _ptr(ws_scale_a), M, N, K, _stream(stream, dev)), "w8a8_linear")
+    return out
+
+
+def w8a8_select_config(M: int, N: int, K: int) -> dict:
+    c = GemmConfig()
+    _check(_lib.w8a8_select_config(M, N, K, ctypes.byref(c)), "w8a8_select_config")
+    return c.as_dict()
+
+
+def w8a8_read_device_error(clear: bool = True) -> int:
+    """Synchronize the device and return (and clear) the kernels' timeout code (0 = none)."""
+    code = ctypes.c_int32(0)
+    st = _lib.w8a8_read_device_error(ctypes.byref(code), 1 if clear else 0)
+    if st not in (W8A8_OK, W8A8_ERR_TIMEOUT):
+        raise W8A8Error(st, "w8a8_read_device_error")
+    return int(code.value)
+
+
+def w8a8_set_wait_timeout_ns(ns: int) -> None:
+    _check(_lib.w8a8_set_wait_timeout_ns(int(ns)), "w8a8_set_wait_timeout_ns")
+
+
+def w8a8_selftest_wait_timeout(timeout_ns: int, stream=None) -> None:
+    _check(_lib.w8a8_selftest_wait_timeout(int(timeout_ns), _stream(stream, torch.device("cuda"))),
+           "w8a8_selftest_wait_timeout")
+
+
+def raw_lib() -> ctypes.CDLL:
+    """The loaded shared object (for tests that call the C ABI with raw pointers)."""
+    return _lib

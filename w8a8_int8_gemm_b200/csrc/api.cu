@@ -1,0 +1,265 @@
+// api.cu -- the C ABI declared in include/w8a8.h: argument validation,
+// per-shape configuration, and the launches.
+//
+// Every argument check happens before any CUDA call, so a rejected call
+// touches no device state and launches nothing.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/w8a8.h"
+#include "internal.h"
+
+namespace w8a8 {
+namespace {
+
+constexpr int64_t kMaxK = 133144;  // K * 127^2 < 2^31
+constexpr int64_t kMaxMN = 2147483647;
+std::atomic<int64_t> g_timeout_ns{2000000000LL};
+
+struct DeviceInfo {
+  bool valid = false;
+  bool supported = false;
+  int sms = 0;
+};
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_dev_mutex;
+
+// Properties of the current device (cached).
+w8a8_status current_device(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return W8A8_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return W8A8_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  DeviceInfo& d = g_devices[dev];
+  if (!d.valid) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      return W8A8_ERR_CUDA;
+    }
+    d.supported = (major == 10 && minor == 0);
+    d.sms = sms;
+    d.valid = true;
+  }
+  *out = d;
+  return d.supported ? W8A8_OK : W8A8_ERR_UNSUPPORTED_DEVICE;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+w8a8_status check_gemm_shape(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || M > kMaxMN || N > kMaxMN) return W8A8_ERR_INVALID_ARG;
+  if (K < 16 || K > kMaxK || K % 16 != 0) return W8A8_ERR_INVALID_ARG;
+  if (N % 8 != 0) return W8A8_ERR_INVALID_ARG;
+  return W8A8_OK;
+}
+
+w8a8_status check_config(const w8a8_gemm_config& c) {
+  if (c.block_m != 128) return W8A8_ERR_INVALID_ARG;
+  if (c.block_n != 128 && c.block_n != 256) return W8A8_ERR_INVALID_ARG;
+  if (c.stages < 2 || c.stages > gemm_max_stages(c.block_n)) return W8A8_ERR_INVALID_ARG;
+  if (c.grid < 1 || c.raster_group < 1) return W8A8_ERR_INVALID_ARG;
+  return W8A8_OK;
+}
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Per-shape choice of the output tile (the paper autotunes its kernel per
+// GEMM shape).  Each persistent CTA does ceil(tiles / SMs) tiles; the cost
+// of a tile is proportional to its column count, with a per-tile overhead
+// (accumulator hand-off, pipeline fill) that favours the wider tile, whose
+// MMAs also read fewer shared-memory bytes per multiply-add.
+w8a8_gemm_config select(int64_t M, int64_t N, int64_t K, int sms) {
+  struct Cand { int bn; double overhead; };
+  const Cand cands[2] = {{256, 0.0}, {128, 0.15}};
+  double best = 1e300;
+  w8a8_gemm_config cfg{};
+  for (const Cand& c : cands) {
+    const int64_t tiles = ceil_div(M, 128) * ceil_div(N, c.bn);
+    const int64_t per_cta = ceil_div(tiles, sms);
+    const double kblocks = static_cast<double>(ceil_div(K, 128));
+    const double cost = static_cast<double>(per_cta) * c.bn * (kblocks + 2.0) * (1.0 + c.overhead);
+    if (cost < best) {
+      best = cost;
+      cfg.block_m = 128;
+      cfg.block_n = c.bn;
+      cfg.stages = gemm_max_stages(c.bn);
+      cfg.grid = static_cast<int>(tiles < sms ? tiles : sms);
+      if (cfg.grid < 1) cfg.grid = 1;
+      cfg.raster_group = 16;
+    }
+  }
+  return cfg;
+}
+
+w8a8_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return W8A8_OK;
+  if (e == cudaErrorInvalidValue) return W8A8_ERR_INVALID_ARG;
+  return W8A8_ERR_LAUNCH;
+}
+
+w8a8_status gemm_common(const int8_t* xq, const int8_t* wq, const float* scale_a, const float* scale_w,
+                        const void* bias, void* out, int64_t M, int64_t N, int64_t K,
+                        const w8a8_gemm_config* user_cfg, GemmOut kind, cudaStream_t stream) {
+  w8a8_status st = check_gemm_shape(M, N, K);
+  if (st != W8A8_OK) return st;
+  if (user_cfg != nullptr && (st = check_config(*user_cfg)) != W8A8_OK) return st;
+  if (M == 0 || N == 0) return W8A8_OK;
+  if (xq == nullptr || wq == nullptr || out == nullptr) return W8A8_ERR_INVALID_ARG;
+  if (kind == GemmOut::kBf16Dequant && (scale_a == nullptr || scale_w == nullptr)) return W8A8_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(wq) || !aligned16(out) || !aligned16(scale_a) || !aligned16(scale_w) ||
+      !aligned16(bias)) {
+    return W8A8_ERR_ALIGNMENT;
+  }
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != W8A8_OK) return st;
+  const w8a8_gemm_config cfg = user_cfg ? *user_cfg : select(M, N, K, dev.sms);
+  GemmArgs a;
+  a.xq = xq;
+  a.wq = wq;
+  a.scale_a = scale_a;
+  a.scale_w = scale_w;
+  a.bias = bias;
+  a.out = out;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.out_kind = kind;
+  a.timeout_ns = static_cast<uint64_t>(g_timeout_ns.load());
+  GemmConfig c{cfg.block_m, cfg.block_n, cfg.stages, cfg.grid, cfg.raster_group};
+  return from_cuda(launch_gemm(a, c, stream));
+}
+
+w8a8_status quantize_common(bool act, const void* x, int64_t M, int64_t K, int64_t ldx, int8_t* xq, int64_t ldxq,
+                            float* scale, cudaStream_t stream) {
+  if (M < 0 || M > kMaxMN || K < 16 || K > kMaxK || K % 16 != 0) return W8A8_ERR_INVALID_ARG;
+  if (ldx < K || ldxq < K) return W8A8_ERR_INVALID_ARG;
+  if (M == 0) return W8A8_OK;
+  if (x == nullptr || xq == nullptr || scale == nullptr) return W8A8_ERR_INVALID_ARG;
+  const int64_t elem = act ? 2 : 4;
+  if (!aligned16(x) || !aligned16(xq) || !aligned16(scale)) return W8A8_ERR_ALIGNMENT;
+  if ((ldx * elem) % 16 != 0 || ldxq % 16 != 0) return W8A8_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  w8a8_status st = current_device(&dev);
+  if (st != W8A8_OK) return st;
+  const cudaError_t e = act ? launch_quantize_act(x, M, K, ldx, xq, ldxq, scale, stream)
+                            : launch_quantize_weight(static_cast<const float*>(x), M, K, ldx, xq, ldxq, scale,
+                                                     stream);
+  return from_cuda(e);
+}
+
+}  // namespace
+}  // namespace w8a8
+
+using namespace w8a8;
+
+extern "C" {
+
+const char* w8a8_status_string(int status) {
+  switch (status) {
+    case W8A8_OK: return "ok";
+    case W8A8_ERR_INVALID_ARG: return "invalid argument";
+    case W8A8_ERR_ALIGNMENT: return "pointer or stride not 16-byte aligned";
+    case W8A8_ERR_UNSUPPORTED_DEVICE: return "device is not sm_100 (B200)";
+    case W8A8_ERR_LAUNCH: return "kernel launch failed";
+    case W8A8_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+    case W8A8_ERR_CUDA: return "CUDA runtime error";
+    default: return "unknown status";
+  }
+}
+
+int w8a8_abi_version(void) { return 100; }
+
+w8a8_status w8a8_quantize_act(const void* x, int64_t M, int64_t K, int64_t ldx, int8_t* xq, int64_t ldxq,
+                              float* scale_a, w8a8_stream_t stream) {
+  return quantize_common(true, x, M, K, ldx, xq, ldxq, scale_a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+w8a8_status w8a8_quantize_weight(const float* w, int64_t N, int64_t K, int64_t ldw, int8_t* wq, int64_t ldwq,
+                                 float* scale_w, w8a8_stream_t stream) {
+  return quantize_common(false, w, N, K, ldw, wq, ldwq, scale_w, reinterpret_cast<cudaStream_t>(stream));
+}
+
+w8a8_status w8a8_gemm(const int8_t* xq, const int8_t* wq, const float* scale_a, const float* scale_w,
+                      const void* bias, void* out, int64_t M, int64_t N, int64_t K, w8a8_stream_t stream) {
+  return gemm_common(xq, wq, scale_a, scale_w, bias, out, M, N, K, nullptr, GemmOut::kBf16Dequant,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+w8a8_status w8a8_gemm_ex(const int8_t* xq, const int8_t* wq, const float* scale_a, const float* scale_w,
+                         const void* bias, void* out, int64_t M, int64_t N, int64_t K,
+                         const w8a8_gemm_config* cfg, w8a8_stream_t stream) {
+  return gemm_common(xq, wq, scale_a, scale_w, bias, out, M, N, K, cfg, GemmOut::kBf16Dequant,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+w8a8_status w8a8_gemm_i32(const int8_t* xq, const int8_t* wq, int32_t* acc, int64_t M, int64_t N, int64_t K,
+                          w8a8_stream_t stream) {
+  return gemm_common(xq, wq, nullptr, nullptr, nullptr, acc, M, N, K, nullptr, GemmOut::kInt32,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+w8a8_status w8a8_gemm_i32_ex(const int8_t* xq, const int8_t* wq, int32_t* acc, int64_t M, int64_t N, int64_t K,
+                             const w8a8_gemm_config* cfg, w8a8_stream_t stream) {
+  return gemm_common(xq, wq, nullptr, nullptr, nullptr, acc, M, N, K, cfg, GemmOut::kInt32,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+w8a8_status w8a8_linear(const void* x, const int8_t* wq, const float* scale_w, const void* bias, void* out,
+                        int8_t* ws_xq, float* ws_scale_a, int64_t M, int64_t N, int64_t K, w8a8_stream_t stream) {
+  // Validate the whole call before launching its first kernel.
+  w8a8_status st = check_gemm_shape(M, N, K);
+  if (st != W8A8_OK) return st;
+  if (M == 0 || N == 0) return W8A8_OK;
+  if (x == nullptr || wq == nullptr || scale_w == nullptr || out == nullptr || ws_xq == nullptr ||
+      ws_scale_a == nullptr) {
+    return W8A8_ERR_INVALID_ARG;
+  }
+  if (!aligned16(x) || !aligned16(wq) || !aligned16(scale_w) || !aligned16(bias) || !aligned16(out) ||
+      !aligned16(ws_xq) || !aligned16(ws_scale_a)) {
+    return W8A8_ERR_ALIGNMENT;
+  }
+  st = w8a8_quantize_act(x, M, K, K, ws_xq, K, ws_scale_a, stream);
+  if (st != W8A8_OK) return st;
+  return w8a8_gemm(ws_xq, wq, ws_scale_a, scale_w, bias, out, M, N, K, stream);
+}
+
+w8a8_status w8a8_select_config(int64_t M, int64_t N, int64_t K, w8a8_gemm_config* cfg) {
+  if (cfg == nullptr) return W8A8_ERR_INVALID_ARG;
+  w8a8_status st = check_gemm_shape(M, N, K);
+  if (st != W8A8_OK) return st;
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != W8A8_OK) return st;
+  *cfg = select(M > 0 ? M : 1, N > 0 ? N : 8, K, dev.sms);
+  return W8A8_OK;
+}
+
+w8a8_status w8a8_read_device_error(int32_t* code, int32_t clear) {
+  if (code == nullptr) return W8A8_ERR_INVALID_ARG;
+  int v = 0;
+  if (read_device_error(&v, clear != 0) != cudaSuccess) return W8A8_ERR_CUDA;
+  *code = v;
+  return v != 0 ? W8A8_ERR_TIMEOUT : W8A8_OK;
+}
+
+w8a8_status w8a8_set_wait_timeout_ns(int64_t ns) {
+  if (ns < 100000) ns = 100000;
+  g_timeout_ns.store(ns);
+  return W8A8_OK;
+}
+
+w8a8_status w8a8_selftest_wait_timeout(int64_t timeout_ns, w8a8_stream_t stream) {
+  if (timeout_ns < 100000) return W8A8_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  w8a8_status st = current_device(&dev);
+  if (st != W8A8_OK) return st;
+  return from_cuda(launch_selftest_wait(static_cast<uint64_t>(timeout_ns), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,501 @@
+// gemm_sm100.cu -- fused W8A8 GEMM for B200 (sm_100a).
+//
+// Paper: "Realizing Native INT8 Compute for Diffusion Transformers on
+// Consumer GPUs" (arXiv 2606.14598), abstract -- an int8 x int8 -> int32
+// GEMM on the tensor cores with the per-token x per-channel dequantization
+// and the bias folded into the epilogue:
+//   out[m,n] = bf16_rne((fl32(acc[m,n]) * scale_a[m]) * scale_w[n] + bias[n]),
+//   acc[m,n] = sum_k xq[m,k] * wq[n,k]  (exact in int32).
+// The paper's kernel is Triton on Ampere mma.sync; this one is written for
+// the 5th-generation tensor cores:
+//
+//   * persistent: one CTA per SM walks output tiles of BLOCK_M x BLOCK_N
+//     (128 x 256 or 128 x 128) in a grouped raster order;
+//   * warp 0 (one elected lane) streams K-slices of 128 bytes of both
+//     operands with TMA into a ring of shared-memory stages (128-byte
+//     swizzle), signalling "full" mbarriers with transaction counts;
+//   * warp 1 allocates tensor memory and (one elected lane) issues
+//     tcgen05.mma.kind::i8, M=128, N=BLOCK_N, K=32 per instruction, into
+//     int32 accumulators held in tensor memory; tcgen05.commit frees each
+//     ring stage when its MMAs retire and marks the accumulator full after
+//     the last K-slice;
+//   * warps 2-5 (the epilogue) each own one 32-lane quarter of tensor
+//     memory (= 32 output rows): they load the int32 accumulators, apply
+//     the dequantization and bias in binary32 in the order above, round to
+//     bf16, stage 32 x 64 bf16 blocks in swizzled shared memory and write
+//     them with TMA stores;
+//   * the accumulator is double-buffered in tensor memory (2 x BLOCK_N
+//     columns), so the epilogue of one tile overlaps the MMAs of the next.
+//
+// Every mbarrier wait is bounded in time (see sm100_ptx.cuh); on timeout the
+// kernel records the site in the device error word, lets its in-flight
+// copies and MMAs finish (again bounded), frees tensor memory and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+namespace w8a8 {
+
+// Device-side error word of this library's kernels (see WaitSite).
+__device__ int g_device_error = 0;
+
+namespace {
+
+constexpr int kBlockM = 128;
+constexpr int kBlockK = 128;            // bytes of K per stage = one 128-byte swizzle row
+constexpr int kMmaK = 32;               // K per tcgen05.mma .kind::i8
+constexpr int kThreads = 192;           // 6 warps
+constexpr int kEpiWarps = 4;
+constexpr int kEpiBufBytes = 32 * 128;  // 32 rows x 128 bytes
+constexpr int kSmemLimit = 232448;      // dynamic shared memory per block on sm_100
+constexpr int kBarrierBytes = 256;
+
+struct Params {
+  int M, N, K;
+  int m_tiles, n_tiles, k_blocks, num_tiles;
+  int raster_group;
+  int stages;
+  const float* scale_a;
+  const float* scale_w;
+  const __nv_bfloat16* bias;
+  uint64_t timeout_ns;
+  int* err;  // device error word
+};
+
+__host__ __device__ constexpr int a_stage_bytes() { return kBlockM * kBlockK; }
+__host__ __device__ constexpr int b_stage_bytes(int bn) { return bn * kBlockK; }
+
+int smem_bytes(int bn, int stages) {
+  return 1024 + stages * (a_stage_bytes() + b_stage_bytes(bn)) + kEpiWarps * 2 * kEpiBufBytes + kBarrierBytes;
+}
+
+__device__ __forceinline__ void tile_coords(int tile, const Params& p, int& mb, int& nb) {
+  const int per_group = p.raster_group * p.n_tiles;
+  const int g = tile / per_group;
+  const int first_m = g * p.raster_group;
+  const int gsz = min(p.raster_group, p.m_tiles - first_m);
+  const int r = tile - g * per_group;
+  mb = first_m + r % gsz;
+  nb = r / gsz;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat16 l = __float2bfloat16_rn(lo);
+  const __nv_bfloat16 h = __float2bfloat16_rn(hi);
+  return static_cast<uint32_t>(__bfloat16_as_ushort(l)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h)) << 16);
+}
+
+// Dequantize 32 accumulators of one row (columns n0 .. n0+31) into 16 packed
+// bf16 pairs: y = (fl32(acc) * sa) * sw[n] + bias[n], each op rounded.
+__device__ __forceinline__ void dequant_32(const uint32_t (&v)[32], float sa, int n0, const Params& p,
+                                           uint32_t* packed) {
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const int n = n0 + 8 * g;
+    float sw[8], bb[8];
+    if (n < p.N) {  // N % 8 == 0: a group of 8 columns is all in or all out
+      const float4 s0 = __ldg(reinterpret_cast<const float4*>(p.scale_w + n));
+      const float4 s1 = __ldg(reinterpret_cast<const float4*>(p.scale_w + n) + 1);
+      sw[0] = s0.x; sw[1] = s0.y; sw[2] = s0.z; sw[3] = s0.w;
+      sw[4] = s1.x; sw[5] = s1.y; sw[6] = s1.z; sw[7] = s1.w;
+      if (p.bias != nullptr) {
+        const uint4 b = __ldg(reinterpret_cast<const uint4*>(p.bias + n));
+        const uint32_t w[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          bb[2 * i] = __uint_as_float(w[i] << 16);
+          bb[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) bb[i] = 0.0f;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { sw[i] = 0.0f; bb[i] = 0.0f; }
+    }
+    float y[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float t = __int2float_rn(static_cast<int>(v[8 * g + i]));
+      t = __fmul_rn(t, sa);
+      t = __fmul_rn(t, sw[i]);
+      y[i] = __fadd_rn(t, bb[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) packed[4 * g + i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
+  }
+}
+
+template <int BN, GemmOut OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                     const __grid_constant__ CUtensorMap tm_d, const Params p) {
+  constexpr uint32_t kA = a_stage_bytes();
+  constexpr uint32_t kB = b_stage_bytes(BN);
+  constexpr uint32_t kTmemCols = 2 * BN;  // two accumulator buffers; 256 or 512 (power of two)
+  constexpr int kColsPerChunk = (OUT == GemmOut::kBf16Dequant) ? 64 : 32;  // 128 output bytes per row
+  constexpr uint32_t kIdesc = make_idesc_i8(kBlockM, BN);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int stages = p.stages;
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + stages * kA;
+  uint8_t* sEpi = sB + stages * kB;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + kEpiWarps * 2 * kEpiBufBytes);
+  uint64_t* empty = full + stages;
+  uint64_t* tfull = empty + stages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&tm_a);
+    prefetch_tensormap(&tm_b);
+    prefetch_tensormap(&tm_d);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish_alloc_permit();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t fills = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      int mb, nb;
+      tile_coords(tile, p, mb, nb);
+      for (int kb = 0; kb < p.k_blocks; ++kb) {
+        ok = warp_wait(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns, p.err, kSiteProducerEmpty);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[stage], kA + kB);
+          tma_load_2d(sA + stage * kA, &tm_a, &full[stage], kb * kBlockK, mb * kBlockM);
+          tma_load_2d(sB + stage * kB, &tm_b, &full[stage], kb * kBlockK, nb * BN);
+        }
+        __syncwarp();
+        ++fills;
+        if (++stage == stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    // Teardown: the last fill of each stage must have landed before the CTA
+    // exits (on the normal path the MMA warp already waited for all of them).
+    if (lane == 0) {
+      const int64_t first = fills > stages ? fills - stages : 0;
+      for (int64_t f = first; f < fills; ++f) {
+        mbar_wait_drain(&full[f % stages], static_cast<uint32_t>((f / stages) & 1), p.timeout_ns, p.err);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int local = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++local) {
+      const int buf = local & 1;
+      const uint32_t tphase = static_cast<uint32_t>(local >> 1) & 1u;
+      ok = warp_wait(&tempty[buf], tphase ^ 1u, abort_flag, p.timeout_ns, p.err, kSiteMmaTmemEmpty);
+      if (!ok) break;
+      tc_fence_after_sync();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+      for (int kb = 0; kb < p.k_blocks; ++kb) {
+        ok = warp_wait(&full[stage], phase, abort_flag, p.timeout_ns, p.err, kSiteMmaFull);
+        if (!ok) break;
+        tc_fence_after_sync();
+        if (lane == 0) {
+          const uint64_t a_desc = make_smem_desc_k_sw128(smem_u32(sA + stage * kA));
+          const uint64_t b_desc = make_smem_desc_k_sw128(smem_u32(sB + stage * kB));
+#pragma unroll
+          for (int k = 0; k < kBlockK / kMmaK; ++k) {
+            // Advance the start address by 32 bytes (2 in units of 16 B)
+            // per K=32 slice inside the 128-byte swizzled row.
+            mma_i8(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc, (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[stage]);
+        }
+        __syncwarp();
+        if (++stage == stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) mma_commit(&tfull[buf]);
+      __syncwarp();
+    }
+    // Teardown: no MMA may still write tensor memory when it is freed.
+    if (lane == 0) {
+      mma_commit(drain);
+      mbar_wait_drain(drain, 0, p.timeout_ns, p.err);
+    }
+    __syncwarp();
+  } else {
+    // --------------------------------------------------------- epilogue
+    const int quarter = warp & 3;  // tensor-memory lanes 32*quarter .. +31
+    const int ew = warp - 2;
+    uint8_t* bufs[2] = {sEpi + (2 * ew) * kEpiBufBytes, sEpi + (2 * ew + 1) * kEpiBufBytes};
+    int local = 0;
+    int nstores = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++local) {
+      int mb, nb;
+      tile_coords(tile, p, mb, nb);
+      const int buf = local & 1;
+      const uint32_t tphase = static_cast<uint32_t>(local >> 1) & 1u;
+      ok = warp_wait(&tfull[buf], tphase, abort_flag, p.timeout_ns, p.err, kSiteEpiTmemFull);
+      if (!ok) break;
+      tc_fence_after_sync();
+
+      const int row0 = mb * kBlockM + quarter * 32;
+      const int row = row0 + lane;
+      float sa = 0.0f;
+      if constexpr (OUT == GemmOut::kBf16Dequant) {
+        if (row < p.M) sa = __ldg(p.scale_a + row);
+      }
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * BN);
+
+#pragma unroll 1
+      for (int c = 0; c < BN / kColsPerChunk; ++c) {
+        const int col0 = nb * BN + c * kColsPerChunk;
+        uint32_t packed[32];
+        if constexpr (OUT == GemmOut::kBf16Dequant) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t v[32];
+            tmem_load_32cols(t_row + c * 64 + h * 32, v);
+            dequant_32(v, sa, col0 + h * 32, p, packed + 16 * h);
+          }
+        } else {
+          uint32_t v[32];
+          tmem_load_32cols(t_row + c * 32, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) packed[i] = v[i];
+        }
+        if (c == BN / kColsPerChunk - 1) {
+          // All of this warp's reads of the accumulator buffer are done.
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);
+        }
+        uint8_t* sb = bufs[nstores & 1];
+        // The store that last read this staging buffer must have finished reading it.
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int pos = j ^ (lane & 7);  // 128-byte swizzle: 16-byte chunk j of row `lane`
+          *reinterpret_cast<uint4*>(sb + lane * 128 + pos * 16) =
+              make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_d, sb, col0, row0);
+          bulk_commit_group();
+        }
+        __syncwarp();
+        ++nstores;
+      }
+    }
+    if (lane == 0) bulk_wait_group<0>();
+    __syncwarp();
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host
+
+// Device address of g_device_error on the current device (looked up once
+// per device; host code must not take the symbol's address directly).
+cudaError_t error_word_address(int** out) {
+  constexpr int kMaxDev = 64;
+  static int* addr[kMaxDev] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_device_error);
+    if (e != cudaSuccess) return e;
+    addr[dev] = static_cast<int*>(p);
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess) {
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows, cols] of `elem` bytes, box [box_rows, box_cols],
+// 128-byte swizzle, zero fill outside the tensor.
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem, const void* base, int64_t rows,
+               int64_t cols, int box_rows, int box_cols) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * static_cast<cuuint64_t>(elem)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, GemmOut OUT>
+cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t stream) {
+  CUtensorMap tm_a, tm_b, tm_d;
+  std::memset(&tm_a, 0, sizeof tm_a);
+  std::memset(&tm_b, 0, sizeof tm_b);
+  std::memset(&tm_d, 0, sizeof tm_d);
+  bool ok = encode_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.xq, a.M, a.K, kBlockM, kBlockK) &&
+            encode_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.wq, a.N, a.K, BN, kBlockK);
+  if constexpr (OUT == GemmOut::kBf16Dequant) {
+    ok = ok && encode_2d(&tm_d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.out, a.M, a.N, 32, 64);
+  } else {
+    ok = ok && encode_2d(&tm_d, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, a.out, a.M, a.N, 32, 32);
+  }
+  if (!ok) return cudaErrorInvalidValue;
+
+  Params p;
+  p.M = static_cast<int>(a.M);
+  p.N = static_cast<int>(a.N);
+  p.K = static_cast<int>(a.K);
+  p.m_tiles = static_cast<int>((a.M + kBlockM - 1) / kBlockM);
+  p.n_tiles = static_cast<int>((a.N + BN - 1) / BN);
+  p.k_blocks = static_cast<int>((a.K + kBlockK - 1) / kBlockK);
+  p.num_tiles = p.m_tiles * p.n_tiles;
+  p.raster_group = cfg.raster_group;
+  p.stages = cfg.stages;
+  p.scale_a = a.scale_a;
+  p.scale_w = a.scale_w;
+  p.bias = static_cast<const __nv_bfloat16*>(a.bias);
+  p.timeout_ns = a.timeout_ns;
+  p.err = nullptr;
+  cudaError_t e = error_word_address(&p.err);
+  if (e != cudaSuccess) return e;
+
+  const int smem = smem_bytes(BN, cfg.stages);
+  auto kernel = gemm_w8a8_kernel<BN, OUT>;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int grid = cfg.grid < p.num_tiles ? cfg.grid : p.num_tiles;
+  kernel<<<grid, kThreads, smem, stream>>>(tm_a, tm_b, tm_d, p);
+  return cudaGetLastError();
+}
+
+__global__ void selftest_wait_kernel(uint64_t timeout_ns, int* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on `bar`: the wait runs out by construction.
+  warp_wait(&bar, 0, &abort_flag, timeout_ns, err, kSiteSelfTest);
+}
+
+}  // namespace
+
+int gemm_max_stages(int block_n) {
+  int s = 0;
+  while (smem_bytes(block_n, s + 1) <= kSmemLimit) ++s;
+  return s;
+}
+
+cudaError_t launch_gemm(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t stream) {
+  const bool bf16 = a.out_kind == GemmOut::kBf16Dequant;
+  if (cfg.block_n == 256) {
+    return bf16 ? launch_typed<256, GemmOut::kBf16Dequant>(a, cfg, stream)
+                : launch_typed<256, GemmOut::kInt32>(a, cfg, stream);
+  }
+  if (cfg.block_n == 128) {
+    return bf16 ? launch_typed<128, GemmOut::kBf16Dequant>(a, cfg, stream)
+                : launch_typed<128, GemmOut::kInt32>(a, cfg, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_selftest_wait(uint64_t timeout_ns, cudaStream_t stream) {
+  int* err = nullptr;
+  cudaError_t e = error_word_address(&err);
+  if (e != cudaSuccess) return e;
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(timeout_ns, err);
+  return cudaGetLastError();
+}
+
+cudaError_t read_device_error(int* value, bool clear) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpyFromSymbol(value, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  if (clear && *value != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero);
+  }
+  return e;
+}
+
+}  // namespace w8a8

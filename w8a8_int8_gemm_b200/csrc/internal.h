@@ -1,0 +1,51 @@
+// internal.h -- launchers shared between the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace w8a8 {
+
+// Tile configuration of the GEMM kernel (see w8a8_gemm_config in w8a8.h).
+struct GemmConfig {
+  int block_m;
+  int block_n;
+  int stages;
+  int grid;
+  int raster_group;
+};
+
+enum class GemmOut { kBf16Dequant = 0, kInt32 = 1 };
+
+struct GemmArgs {
+  const int8_t* xq;
+  const int8_t* wq;
+  const float* scale_a;
+  const float* scale_w;
+  const void* bias;  // bf16 [N] or nullptr
+  void* out;         // bf16 [M, N] or int32 [M, N]
+  int64_t M, N, K;
+  GemmOut out_kind;
+  uint64_t timeout_ns;
+};
+
+cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq,
+                                float* scale, cudaStream_t stream);
+cudaError_t launch_quantize_weight(const float* w, int64_t N, int64_t K, int64_t ldw, int8_t* q, int64_t ldq,
+                                   float* scale, cudaStream_t stream);
+
+// Largest stage count the shared memory holds for a block_n (0 if none).
+int gemm_max_stages(int block_n);
+
+// Returns cudaSuccess or the launch error; tensor-map encoding failures are
+// reported as cudaErrorInvalidValue.
+cudaError_t launch_gemm(const GemmArgs& args, const GemmConfig& cfg, cudaStream_t stream);
+
+cudaError_t launch_selftest_wait(uint64_t timeout_ns, cudaStream_t stream);
+
+// Synchronizes the current device and reads (optionally clears) the device
+// error word written by timed-out waits.
+cudaError_t read_device_error(int* value, bool clear);
+
+}  // namespace w8a8
