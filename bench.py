@@ -332,7 +332,7 @@ def run_native(args, wl) -> None:
 
     result = None
     if rank == 0:
-        e2e = run_e2e(w8, wl, x_host, sets[0]["wq"], sw, bias, dev, stream, args)
+        e2e = run_e2e(w8, wl, x_host, sets[0]["wq"], sw, bias, dev, stream, args) if args.e2e_steps else None
         ctx = context_baselines(wl, d, sets[0], sw, bias, dev, args) if not args.no_context else None
         cpu = cpu_baseline(wl) if (world == 1 and not args.no_cpu_baseline) else None
         cfg = wl_config(wl)

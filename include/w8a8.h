@@ -145,10 +145,11 @@ W8A8_API w8a8_status w8a8_gemm_i32(const int8_t* xq, const int8_t* wq, int32_t* 
  * shape"; here a static cost model over a measured table of tile shapes).
  */
 typedef struct {
-    int32_t block_m;       /* rows of the output tile per CTA: 128 */
+    int32_t block_m;       /* rows of the output tile: 128 (one CTA) or 256 (a CTA pair
+                              sharing each MMA through tcgen05 cta_group::2) */
     int32_t block_n;       /* columns of the output tile: 128 or 256 */
     int32_t stages;        /* depth of the shared-memory operand ring */
-    int32_t grid;          /* persistent CTAs launched (<= number of SMs) */
+    int32_t grid;          /* persistent CTAs launched (<= number of SMs; even for pairs) */
     int32_t raster_group;  /* M tiles walked together before moving along N */
     int32_t reserved[3];   /* zero */
 } w8a8_gemm_config;
@@ -158,10 +159,11 @@ typedef struct {
 W8A8_API w8a8_status w8a8_select_config(int64_t M, int64_t N, int64_t K, w8a8_gemm_config* cfg);
 
 /* w8a8_gemm / w8a8_gemm_i32 with an explicit configuration (cfg NULL means
- * the selected one).  block_m must be 128, block_n 128 or 256, stages within
- * what shared memory holds (2..4 at block_n 256, 2..6 at 128), 1 <= grid,
- * 1 <= raster_group; anything else is W8A8_ERR_INVALID_ARG.  For sweeps and
- * tests: every valid configuration computes the same result. */
+ * the selected one).  block_m 128 or 256, block_n 128 or 256, stages from 2
+ * to what shared memory holds (4 at 128 x 256, 6 at 128 x 128 and 256 x 256,
+ * 8 at 256 x 128), grid >= 1 (>= 2 for block_m 256), raster_group >= 1;
+ * anything else is W8A8_ERR_INVALID_ARG.  For sweeps and tests: every valid
+ * configuration computes the same result. */
 W8A8_API w8a8_status w8a8_gemm_ex(const int8_t* xq, const int8_t* wq, const float* scale_a,
                          const float* scale_w, const void* bias, void* out,
                          int64_t M, int64_t N, int64_t K, const w8a8_gemm_config* cfg,

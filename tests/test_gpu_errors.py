@@ -53,7 +53,9 @@ def test_rejects_bad_config(w8):
                 dict(block_m=128, block_n=192, stages=4, grid=1, raster_group=1),
                 dict(block_m=128, block_n=256, stages=5, grid=1, raster_group=1),
                 dict(block_m=128, block_n=128, stages=1, grid=1, raster_group=1),
-                dict(block_m=128, block_n=128, stages=2, grid=0, raster_group=1)]:
+                dict(block_m=128, block_n=128, stages=2, grid=0, raster_group=1),
+                dict(block_m=256, block_n=256, stages=7, grid=2, raster_group=1),
+                dict(block_m=256, block_n=256, stages=4, grid=1, raster_group=1)]:
         with pytest.raises(w8.W8A8Error):
             w8.w8a8_gemm_i32(xq, wq, config=cfg)
 

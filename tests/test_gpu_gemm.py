@@ -36,7 +36,8 @@ def _i32(w8, xq, wq, config=None):
     return acc.cpu().numpy().astype(np.int64)
 
 
-SHAPES = [(1, 8, 16), (63, 136, 48), (129, 264, 272), (64, 128, 256), (200, 520, 400), (257, 256, 1040)]
+SHAPES = [(1, 8, 16), (63, 136, 48), (129, 264, 272), (64, 128, 256), (200, 520, 400), (257, 256, 1040),
+          (384, 392, 144), (520, 776, 2064)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
@@ -46,12 +47,17 @@ def test_i32_ragged_shapes(w8, M, N, K):
     assert np.array_equal(_i32(w8, xq, wq), oracle.gemm_i64(xq, wq))
 
 
-CONFIGS = [dict(block_m=128, block_n=bn, stages=st, grid=g, raster_group=rg)
-           for bn, st in [(256, 4), (256, 2), (256, 3), (128, 6), (128, 2), (128, 4)]
-           for g, rg in [(148, 16), (3, 1), (1, 5)]]
+CONFIGS = [dict(block_m=bm, block_n=bn, stages=st, grid=g, raster_group=rg)
+           for bm, bn, st in [(128, 256, 4), (128, 256, 2), (128, 128, 6), (128, 128, 3),
+                              (256, 256, 6), (256, 256, 2), (256, 128, 8), (256, 128, 3)]
+           for g, rg in [(148, 16), (4, 1), (2, 5)]]
 
 
-@pytest.mark.parametrize("cfg", CONFIGS, ids=lambda c: f"bn{c['block_n']}_st{c['stages']}_g{c['grid']}_r{c['raster_group']}")
+def _cid(c):
+    return f"m{c['block_m']}_n{c['block_n']}_st{c['stages']}_g{c['grid']}_r{c['raster_group']}"
+
+
+@pytest.mark.parametrize("cfg", CONFIGS, ids=_cid)
 def test_i32_every_config(w8, cfg):
     rng = np.random.default_rng(cfg["block_n"] + cfg["stages"] * 10 + cfg["grid"])
     M, N, K = 300, 776, 656
@@ -125,7 +131,7 @@ def test_bf16_epilogue(w8, M, N, K, bias):
     assert bf16_ulp_diff(got, want).max() <= 1
 
 
-@pytest.mark.parametrize("cfg", CONFIGS[::3], ids=lambda c: f"bn{c['block_n']}_st{c['stages']}")
+@pytest.mark.parametrize("cfg", CONFIGS[::3], ids=_cid)
 def test_bf16_epilogue_configs(w8, cfg):
     got, want = _bf16_gemm_case(w8, 300, 776, 656, cfg["block_n"] + cfg["stages"], True, cfg)
     assert bf16_ulp_diff(got, want).max() <= 1
@@ -157,5 +163,5 @@ def test_empty_problem(w8):
 def test_selected_configs_valid(w8):
     for name, wl in workloads.WORKLOADS.items():
         c = w8.w8a8_select_config(wl.M, wl.N, wl.K)
-        assert c["block_m"] == 128 and c["block_n"] in (128, 256), (name, c)
+        assert c["block_m"] in (128, 256) and c["block_n"] in (128, 256), (name, c)
         assert 1 <= c["grid"] <= torch.cuda.get_device_properties(0).multi_processor_count

@@ -8,8 +8,9 @@ benchmark uses (the selected tile configuration, all tokens in one call):
 * the bf16 output is within 1 ulp of the oracle on sampled rows (first,
   last, tile-boundary and random rows) -- the oracle's exact GEMM on every
   row of the large shapes would take minutes of CPU -- and has no NaN;
-* the cosine similarity with the unquantized fp64 product is reported and
-  must be high (the paper reports cosine 1.0 for its kernel).
+* cosine similarity (the paper's accuracy metric): against the fp64 product
+  of the dequantized operands it is 1 up to bf16 output rounding; against
+  the unquantized fp64 product it must stay high.
 
 Paper: "Realizing Native INT8 Compute for Diffusion Transformers on Consumer
 GPUs" (arXiv 2606.14598), abstract."""
@@ -59,12 +60,24 @@ def _run(w8, name, n_sample):
     ulp = bf16_ulp_diff(got[rows], out_o)
     assert ulp.max() <= 1, f"max {ulp.max()} ulp at {np.argwhere(ulp > 1)[:3].tolist()}"
 
-    # the paper's accuracy metric, against the unquantized product
-    xf = oracle.bf16_bits_to_f32(d["x"][rows[:8]]).astype(np.float64)
-    ref = xf @ d["w"].astype(np.float64).T + oracle.bf16_bits_to_f32(d["bias"]).astype(np.float64)
-    y = torch.from_numpy(got[rows[:8]].view(np.int16)).view(torch.bfloat16).double().numpy()
-    cos = float((ref * y).sum() / np.sqrt((ref * ref).sum() * (y * y).sum()))
-    assert cos > 0.999, cos
+    # The paper's accuracy metric (cosine similarity).  Against the product of
+    # the dequantized operands (xq*s_a)(wq*s_w)^T + bias in fp64 only the bf16
+    # output rounding separates the two: cosine >= 1 - 2^-15.  Against the
+    # unquantized fp64 product the int8 quantization error enters too; for
+    # the outlier workload (per-token step ~ 20*max|N(0,1)|/127) it is about
+    # 1e-3, so that check only guards against gross errors.
+    r8 = rows[:8]
+    y = torch.from_numpy(got[r8].view(np.int16)).view(torch.bfloat16).double().numpy()
+    b64 = oracle.bf16_bits_to_f32(d["bias"]).astype(np.float64)
+    deq = (xq_o[r8].astype(np.float64) * sa_o[r8, None]) @ (wq_o.astype(np.float64) * sw_o[:, None]).T + b64
+    xf = oracle.bf16_bits_to_f32(d["x"][r8]).astype(np.float64)
+    ref = xf @ d["w"].astype(np.float64).T + b64
+
+    def cos(a, b):
+        return float((a * b).sum() / np.sqrt((a * a).sum() * (b * b).sum()))
+
+    assert cos(deq, y) >= 1 - 2.0 ** -15, cos(deq, y)
+    assert cos(ref, y) >= 0.99, cos(ref, y)
     return ulp
 
 

@@ -61,38 +61,42 @@ w8a8_status check_gemm_shape(int64_t M, int64_t N, int64_t K) {
 }
 
 w8a8_status check_config(const w8a8_gemm_config& c) {
-  if (c.block_m != 128) return W8A8_ERR_INVALID_ARG;
+  if (c.block_m != 128 && c.block_m != 256) return W8A8_ERR_INVALID_ARG;
   if (c.block_n != 128 && c.block_n != 256) return W8A8_ERR_INVALID_ARG;
-  if (c.stages < 2 || c.stages > gemm_max_stages(c.block_n)) return W8A8_ERR_INVALID_ARG;
-  if (c.grid < 1 || c.raster_group < 1) return W8A8_ERR_INVALID_ARG;
+  if (c.stages < 2 || c.stages > gemm_max_stages(c.block_m, c.block_n)) return W8A8_ERR_INVALID_ARG;
+  if (c.grid < (c.block_m == 256 ? 2 : 1) || c.raster_group < 1) return W8A8_ERR_INVALID_ARG;
   return W8A8_OK;
 }
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Per-shape choice of the output tile (the paper autotunes its kernel per
-// GEMM shape).  Each persistent CTA does ceil(tiles / SMs) tiles; the cost
-// of a tile is proportional to its column count, with a per-tile overhead
-// (accumulator hand-off, pipeline fill) that favours the wider tile, whose
-// MMAs also read fewer shared-memory bytes per multiply-add.
+// GEMM shape).  Candidates: 256 x 256 and 256 x 128 tiles computed by CTA
+// pairs (cta_group::2; each SM stages half of B, so more ring stages fit and
+// less operand traffic flows per multiply-add), and 128 x 256 / 128 x 128
+// tiles on single CTAs for short M.  Each persistent CTA (pair) does
+// ceil(tiles / units) tiles; a tile costs its area times (K blocks + a
+// fixed per-tile overhead), scaled by the shape's relative efficiency.
 w8a8_gemm_config select(int64_t M, int64_t N, int64_t K, int sms) {
-  struct Cand { int bn; double overhead; };
-  const Cand cands[2] = {{256, 0.0}, {128, 0.15}};
+  struct Cand { int bm, bn; double rel_cost; };
+  const Cand cands[4] = {{256, 256, 1.00}, {256, 128, 1.08}, {128, 256, 1.30}, {128, 128, 1.45}};
   double best = 1e300;
   w8a8_gemm_config cfg{};
+  const double kblocks = static_cast<double>(ceil_div(K, 128));
   for (const Cand& c : cands) {
-    const int64_t tiles = ceil_div(M, 128) * ceil_div(N, c.bn);
-    const int64_t per_cta = ceil_div(tiles, sms);
-    const double kblocks = static_cast<double>(ceil_div(K, 128));
-    const double cost = static_cast<double>(per_cta) * c.bn * (kblocks + 2.0) * (1.0 + c.overhead);
+    const int units = c.bm == 256 ? sms / 2 : sms;
+    const int64_t tiles = ceil_div(M, c.bm) * ceil_div(N, c.bn);
+    const int64_t per_unit = ceil_div(tiles, units);
+    const double cost = static_cast<double>(per_unit) * c.bm * c.bn * (kblocks + 2.0) * c.rel_cost /
+                        (c.bm == 256 ? 2.0 : 1.0);
     if (cost < best) {
       best = cost;
-      cfg.block_m = 128;
+      cfg.block_m = c.bm;
       cfg.block_n = c.bn;
-      cfg.stages = gemm_max_stages(c.bn);
-      cfg.grid = static_cast<int>(tiles < sms ? tiles : sms);
-      if (cfg.grid < 1) cfg.grid = 1;
-      cfg.raster_group = 16;
+      cfg.stages = gemm_max_stages(c.bm, c.bn);
+      const int64_t used = tiles < units ? tiles : units;
+      cfg.grid = static_cast<int>(used * (c.bm == 256 ? 2 : 1));
+      cfg.raster_group = 8;
     }
   }
   return cfg;

@@ -70,10 +70,13 @@ struct Params {
 };
 
 __host__ __device__ constexpr int a_stage_bytes() { return kBlockM * kBlockK; }
-__host__ __device__ constexpr int b_stage_bytes(int bn) { return bn * kBlockK; }
 
-int smem_bytes(int bn, int stages) {
-  return 1024 + stages * (a_stage_bytes() + b_stage_bytes(bn)) + kEpiWarps * 2 * kEpiBufBytes + kBarrierBytes;
+// Dynamic shared memory of one CTA: alignment slack, the operand ring (A:
+// 128 rows, B: block_n rows, or block_n / 2 for a CTA pair), the epilogue's
+// staging buffers and the barriers.
+int smem_bytes(bool pair, int bn, int stages) {
+  const int b_rows = pair ? bn / 2 : bn;
+  return 1024 + stages * (a_stage_bytes() + b_rows * kBlockK) + kEpiWarps * 2 * kEpiBufBytes + kBarrierBytes;
 }
 
 __device__ __forceinline__ void tile_coords(int tile, const Params& p, int& mb, int& nb) {
@@ -134,15 +137,28 @@ __device__ __forceinline__ void dequant_32(const uint32_t (&v)[32], float sa, in
   }
 }
 
-template <int BN, GemmOut OUT>
+// One kernel for both tile shapes.  PAIR = false: one CTA computes a
+// 128 x BN tile.  PAIR = true: a cluster of two CTAs computes a 256 x BN tile
+// with tcgen05 cta_group::2 -- each CTA loads its own 128 rows of A and half
+// (BN/2 rows) of B, the pair's leader (cluster rank 0) issues M=256 MMAs that
+// read both CTAs' shared memory, and each CTA's tensor memory receives its
+// own 128 rows of the accumulator.  Barriers of the pair: the leader's "full"
+// stages count both CTAs' TMA bytes; the leader's commits arrive on the
+// "empty" and "accumulator full" barriers of both CTAs; both CTAs' epilogue
+// warps arrive on the leader's "accumulator empty" barrier.
+template <int BN, GemmOut OUT, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_d, const Params p) {
+  constexpr int kTileM = PAIR ? 2 * kBlockM : kBlockM;  // rows of the output tile
+  constexpr int kBRows = PAIR ? BN / 2 : BN;             // rows of B this CTA loads
   constexpr uint32_t kA = a_stage_bytes();
-  constexpr uint32_t kB = b_stage_bytes(BN);
+  constexpr uint32_t kB = kBRows * kBlockK;
+  constexpr uint32_t kTxBytes = (PAIR ? 2 : 1) * (kA + kB);
   constexpr uint32_t kTmemCols = 2 * BN;  // two accumulator buffers; 256 or 512 (power of two)
   constexpr int kColsPerChunk = (OUT == GemmOut::kBf16Dequant) ? 64 : 32;  // 128 output bytes per row
-  constexpr uint32_t kIdesc = make_idesc_i8(kBlockM, BN);
+  constexpr uint32_t kIdesc = make_idesc_i8(kTileM, BN);
+  constexpr int kEpiArrivals = (PAIR ? 2 : 1) * kEpiWarps;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -160,6 +176,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = (rank == 0);
+  // Tiles are walked per CTA (single) or per CTA pair.
+  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int num_units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
@@ -168,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], kEpiWarps);
+      mbar_init(&tempty[b], kEpiArrivals);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -177,14 +198,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tm_b);
     prefetch_tensormap(&tm_d);
   }
+  if constexpr (PAIR) {
+    cluster_sync_all();  // the peer's barriers exist before anyone signals them
+  } else {
+    __syncthreads();
+  }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish_alloc_permit();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, kTmemCols);
+      tmem_relinquish_alloc_permit_pair();
+    } else {
+      tmem_alloc(tmem_slot, kTmemCols);
+      tmem_relinquish_alloc_permit();
+    }
   }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  const uint32_t peer_abort = PAIR ? map_to_cta(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u) : 0u;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
@@ -192,16 +224,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t phase = 0;
     int64_t fills = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+    for (int tile = unit; ok && tile < p.num_tiles; tile += num_units) {
       int mb, nb;
       tile_coords(tile, p, mb, nb);
+      const int a_row = mb * kTileM + static_cast<int>(rank) * kBlockM;
+      const int b_row = nb * BN + static_cast<int>(rank) * kBRows;
       for (int kb = 0; kb < p.k_blocks; ++kb) {
         ok = warp_wait(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns, p.err, kSiteProducerEmpty);
         if (!ok) break;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full[stage], kA + kB);
-          tma_load_2d(sA + stage * kA, &tm_a, &full[stage], kb * kBlockK, mb * kBlockM);
-          tma_load_2d(sB + stage * kB, &tm_b, &full[stage], kb * kBlockK, nb * BN);
+          if constexpr (PAIR) {
+            const uint32_t bar = map_to_cta(smem_u32(&full[stage]), 0u);
+            if (leader) mbar_arrive_expect_tx(&full[stage], kTxBytes);
+            tma_load_2d_pair(sA + stage * kA, &tm_a, bar, kb * kBlockK, a_row);
+            tma_load_2d_pair(sB + stage * kB, &tm_b, bar, kb * kBlockK, b_row);
+          } else {
+            mbar_arrive_expect_tx(&full[stage], kTxBytes);
+            tma_load_2d(sA + stage * kA, &tm_a, &full[stage], kb * kBlockK, a_row);
+            tma_load_2d(sB + stage * kB, &tm_b, &full[stage], kb * kBlockK, b_row);
+          }
         }
         __syncwarp();
         ++fills;
@@ -211,9 +252,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    if (!ok && PAIR && lane == 0) st_cluster_u32(peer_abort, 1u);
     // Teardown: the last fill of each stage must have landed before the CTA
-    // exits (on the normal path the MMA warp already waited for all of them).
-    if (lane == 0) {
+    // exits (on the normal path the MMA warp already waited for all of
+    // them).  A pair's loads complete on the leader's barriers, which the
+    // leader drains for both CTAs.
+    if (leader && lane == 0) {
       const int64_t first = fills > stages ? fills - stages : 0;
       for (int64_t f = first; f < fills; ++f) {
         mbar_wait_drain(&full[f % stages], static_cast<uint32_t>((f / stages) & 1), p.timeout_ns, p.err);
@@ -222,48 +266,72 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
-    int stage = 0;
-    uint32_t phase = 0;
-    int local = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++local) {
-      const int buf = local & 1;
-      const uint32_t tphase = static_cast<uint32_t>(local >> 1) & 1u;
-      ok = warp_wait(&tempty[buf], tphase ^ 1u, abort_flag, p.timeout_ns, p.err, kSiteMmaTmemEmpty);
-      if (!ok) break;
-      tc_fence_after_sync();
-      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
-      for (int kb = 0; kb < p.k_blocks; ++kb) {
-        ok = warp_wait(&full[stage], phase, abort_flag, p.timeout_ns, p.err, kSiteMmaFull);
+    if (leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int tile = unit; ok && tile < p.num_tiles; tile += num_units, ++local) {
+        const int buf = local & 1;
+        const uint32_t tphase = static_cast<uint32_t>(local >> 1) & 1u;
+        ok = warp_wait(&tempty[buf], tphase ^ 1u, abort_flag, p.timeout_ns, p.err, kSiteMmaTmemEmpty);
         if (!ok) break;
         tc_fence_after_sync();
-        if (lane == 0) {
-          const uint64_t a_desc = make_smem_desc_k_sw128(smem_u32(sA + stage * kA));
-          const uint64_t b_desc = make_smem_desc_k_sw128(smem_u32(sB + stage * kB));
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          ok = warp_wait(&full[stage], phase, abort_flag, p.timeout_ns, p.err, kSiteMmaFull);
+          if (!ok) break;
+          tc_fence_after_sync();
+          if (lane == 0) {
+            const uint64_t a_desc = make_smem_desc_k_sw128(smem_u32(sA + stage * kA));
+            const uint64_t b_desc = make_smem_desc_k_sw128(smem_u32(sB + stage * kB));
 #pragma unroll
-          for (int k = 0; k < kBlockK / kMmaK; ++k) {
-            // Advance the start address by 32 bytes (2 in units of 16 B)
-            // per K=32 slice inside the 128-byte swizzled row.
-            mma_i8(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc, (kb > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < kBlockK / kMmaK; ++k) {
+              // Advance the start address by 32 bytes (2 in units of 16 B)
+              // per K=32 slice inside the 128-byte swizzled row.
+              const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+              if constexpr (PAIR) {
+                mma_i8_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc, acc);
+              } else {
+                mma_i8(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc, acc);
+              }
+            }
+            if constexpr (PAIR) {
+              mma_commit_pair(smem_u32(&empty[stage]));
+              mma_commit_pair(map_to_cta(smem_u32(&empty[stage]), 1u));
+            } else {
+              mma_commit(&empty[stage]);
+            }
           }
-          mma_commit(&empty[stage]);
+          __syncwarp();
+          if (++stage == stages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        if (lane == 0) {
+          if constexpr (PAIR) {
+            mma_commit_pair(smem_u32(&tfull[buf]));
+            mma_commit_pair(map_to_cta(smem_u32(&tfull[buf]), 1u));
+          } else {
+            mma_commit(&tfull[buf]);
+          }
         }
         __syncwarp();
-        if (++stage == stages) {
-          stage = 0;
-          phase ^= 1u;
-        }
       }
-      if (!ok) break;
-      if (lane == 0) mma_commit(&tfull[buf]);
+      if (!ok && PAIR && lane == 0) st_cluster_u32(peer_abort, 1u);
+      // Teardown: no MMA may still write tensor memory when it is freed.
+      if (lane == 0) {
+        if constexpr (PAIR) {
+          mma_commit_pair(smem_u32(drain));
+        } else {
+          mma_commit(drain);
+        }
+        mbar_wait_drain(drain, 0, p.timeout_ns, p.err);
+      }
       __syncwarp();
     }
-    // Teardown: no MMA may still write tensor memory when it is freed.
-    if (lane == 0) {
-      mma_commit(drain);
-      mbar_wait_drain(drain, 0, p.timeout_ns, p.err);
-    }
-    __syncwarp();
   } else {
     // --------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // tensor-memory lanes 32*quarter .. +31
@@ -272,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int local = 0;
     int nstores = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++local) {
+    for (int tile = unit; ok && tile < p.num_tiles; tile += num_units, ++local) {
       int mb, nb;
       tile_coords(tile, p, mb, nb);
       const int buf = local & 1;
@@ -281,13 +349,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after_sync();
 
-      const int row0 = mb * kBlockM + quarter * 32;
+      const int row0 = mb * kTileM + static_cast<int>(rank) * kBlockM + quarter * 32;
       const int row = row0 + lane;
       float sa = 0.0f;
       if constexpr (OUT == GemmOut::kBf16Dequant) {
         if (row < p.M) sa = __ldg(p.scale_a + row);
       }
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * BN);
+      const uint32_t t_row =
+          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * BN);
 
 #pragma unroll 1
       for (int c = 0; c < BN / kColsPerChunk; ++c) {
@@ -310,8 +379,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           // All of this warp's reads of the accumulator buffer are done.
           tc_fence_before_sync();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[buf]);
+          if (lane == 0) {
+            if (PAIR && !leader) {
+              mbar_arrive_cluster(map_to_cta(smem_u32(&tempty[buf]), 0u));
+            } else {
+              mbar_arrive(&tempty[buf]);
+            }
+          }
         }
+        if (row0 >= p.M || col0 >= p.N) continue;  // block entirely outside the output
         uint8_t* sb = bufs[nstores & 1];
         // The store that last read this staging buffer must have finished reading it.
         if (lane == 0) bulk_wait_group_read<1>();
@@ -332,15 +408,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++nstores;
       }
     }
+    if (!ok && PAIR && lane == 0) st_cluster_u32(peer_abort, 1u);
     if (lane == 0) bulk_wait_group<0>();
     __syncwarp();
   }
 
   tc_fence_before_sync();
   __syncthreads();
+  if (*abort_flag) {
+    // A wait ran out somewhere: give copies already issued (by this CTA or
+    // its peer, whose loads signal the leader) time to land before the
+    // shared memory they target is released.
+    if (threadIdx.x == 0) {
+      const uint64_t t0 = global_timer_ns();
+      while (global_timer_ns() - t0 < 200000ull) {
+      }
+    }
+    __syncthreads();
+  }
+  if constexpr (PAIR) cluster_sync_all();
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if constexpr (PAIR) {
+      tmem_dealloc_pair(tmem_base, kTmemCols);
+    } else {
+      tmem_dealloc(tmem_base, kTmemCols);
+    }
   }
 }
 
@@ -402,14 +495,16 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem, const void
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, GemmOut OUT>
+template <int BN, GemmOut OUT, bool PAIR>
 cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t stream) {
+  constexpr int kTileM = PAIR ? 2 * kBlockM : kBlockM;
+  constexpr int kBRows = PAIR ? BN / 2 : BN;
   CUtensorMap tm_a, tm_b, tm_d;
   std::memset(&tm_a, 0, sizeof tm_a);
   std::memset(&tm_b, 0, sizeof tm_b);
   std::memset(&tm_d, 0, sizeof tm_d);
   bool ok = encode_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.xq, a.M, a.K, kBlockM, kBlockK) &&
-            encode_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.wq, a.N, a.K, BN, kBlockK);
+            encode_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.wq, a.N, a.K, kBRows, kBlockK);
   if constexpr (OUT == GemmOut::kBf16Dequant) {
     ok = ok && encode_2d(&tm_d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.out, a.M, a.N, 32, 64);
   } else {
@@ -421,7 +516,7 @@ cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t 
   p.M = static_cast<int>(a.M);
   p.N = static_cast<int>(a.N);
   p.K = static_cast<int>(a.K);
-  p.m_tiles = static_cast<int>((a.M + kBlockM - 1) / kBlockM);
+  p.m_tiles = static_cast<int>((a.M + kTileM - 1) / kTileM);
   p.n_tiles = static_cast<int>((a.N + BN - 1) / BN);
   p.k_blocks = static_cast<int>((a.K + kBlockK - 1) / kBlockK);
   p.num_tiles = p.m_tiles * p.n_tiles;
@@ -435,12 +530,29 @@ cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t 
   cudaError_t e = error_word_address(&p.err);
   if (e != cudaSuccess) return e;
 
-  const int smem = smem_bytes(BN, cfg.stages);
-  auto kernel = gemm_w8a8_kernel<BN, OUT>;
+  const int smem = smem_bytes(PAIR, BN, cfg.stages);
+  auto kernel = gemm_w8a8_kernel<BN, OUT, PAIR>;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const int grid = cfg.grid < p.num_tiles ? cfg.grid : p.num_tiles;
-  kernel<<<grid, kThreads, smem, stream>>>(tm_a, tm_b, tm_d, p);
+  // Persistent grid: one CTA (or CTA pair) per tile at most.
+  int units = (PAIR ? cfg.grid / 2 : cfg.grid);
+  if (units < 1) units = 1;
+  if (units > p.num_tiles) units = p.num_tiles;
+  cudaLaunchConfig_t lc;
+  std::memset(&lc, 0, sizeof lc);
+  lc.gridDim = dim3(static_cast<unsigned>(units * (PAIR ? 2 : 1)));
+  lc.blockDim = dim3(kThreads);
+  lc.dynamicSmemBytes = static_cast<size_t>(smem);
+  lc.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = PAIR ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  e = cudaLaunchKernelEx(&lc, kernel, tm_a, tm_b, tm_d, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -459,21 +571,34 @@ __global__ void selftest_wait_kernel(uint64_t timeout_ns, int* err) {
 
 }  // namespace
 
-int gemm_max_stages(int block_n) {
+int gemm_max_stages(int block_m, int block_n) {
+  const bool pair = block_m == 2 * kBlockM;
   int s = 0;
-  while (smem_bytes(block_n, s + 1) <= kSmemLimit) ++s;
+  while (smem_bytes(pair, block_n, s + 1) <= kSmemLimit) ++s;
   return s;
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t stream) {
   const bool bf16 = a.out_kind == GemmOut::kBf16Dequant;
-  if (cfg.block_n == 256) {
-    return bf16 ? launch_typed<256, GemmOut::kBf16Dequant>(a, cfg, stream)
-                : launch_typed<256, GemmOut::kInt32>(a, cfg, stream);
-  }
-  if (cfg.block_n == 128) {
-    return bf16 ? launch_typed<128, GemmOut::kBf16Dequant>(a, cfg, stream)
-                : launch_typed<128, GemmOut::kInt32>(a, cfg, stream);
+  using O = GemmOut;
+  if (cfg.block_m == 256) {
+    if (cfg.block_n == 256) {
+      return bf16 ? launch_typed<256, O::kBf16Dequant, true>(a, cfg, stream)
+                  : launch_typed<256, O::kInt32, true>(a, cfg, stream);
+    }
+    if (cfg.block_n == 128) {
+      return bf16 ? launch_typed<128, O::kBf16Dequant, true>(a, cfg, stream)
+                  : launch_typed<128, O::kInt32, true>(a, cfg, stream);
+    }
+  } else if (cfg.block_m == 128) {
+    if (cfg.block_n == 256) {
+      return bf16 ? launch_typed<256, O::kBf16Dequant, false>(a, cfg, stream)
+                  : launch_typed<256, O::kInt32, false>(a, cfg, stream);
+    }
+    if (cfg.block_n == 128) {
+      return bf16 ? launch_typed<128, O::kBf16Dequant, false>(a, cfg, stream)
+                  : launch_typed<128, O::kInt32, false>(a, cfg, stream);
+    }
   }
   return cudaErrorInvalidValue;
 }

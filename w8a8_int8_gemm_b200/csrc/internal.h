@@ -35,8 +35,9 @@ cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int64_t ldx
 cudaError_t launch_quantize_weight(const float* w, int64_t N, int64_t K, int64_t ldw, int8_t* q, int64_t ldq,
                                    float* scale, cudaStream_t stream);
 
-// Largest stage count the shared memory holds for a block_n (0 if none).
-int gemm_max_stages(int block_n);
+// Largest stage count the shared memory holds for a tile shape (0 if none).
+// block_m 128: one CTA per tile; block_m 256: a CTA pair (cluster of 2).
+int gemm_max_stages(int block_m, int block_n);
 
 // Returns cudaSuccess or the launch error; tensor-map encoding failures are
 // reported as cudaErrorInvalidValue.

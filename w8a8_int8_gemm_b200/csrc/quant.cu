@@ -8,22 +8,24 @@
 //   scale[r] = fl32(max_k |x[r,k]| / 127)
 //   q[r,k]   = clamp(rne(fl32(x[r,k] / scale[r])), -127, 127), 0 if scale[r] == 0
 //
-// Layout: one warp per row.  Lanes read 16-byte vectors (8 bf16 or 4 fp32),
-// keep up to VPL of them in registers, reduce |x| with a butterfly shuffle,
-// then write the packed int8 codes (8 or 4 bytes per lane per vector).  The
-// kernel moves 3 bytes per bf16 element (2 in, 1 out) and is bound by HBM
-// bandwidth.
+// Layout: one warp per row, all rows in flight at once (about 40 registers
+// per thread, 48 warps per SM).  Pass 1 reads the row as 16-byte vectors
+// (8 bf16 or 4 fp32), four per lane in flight, and reduces |x| with a
+// butterfly shuffle; pass 2 reads the row again -- from L1, where pass 1
+// left it -- and writes the packed int8 codes (8 or 4 bytes per lane per
+// vector).  HBM sees 3 bytes per bf16 element (2 in, 1 out): the kernel is
+// bound by HBM bandwidth.
 //
 // Exactness.  The code q is decided in binary32 exactly as the definition
 // says.  Instead of one IEEE division per element, the kernel multiplies by
 // the row's reciprocal r = fl32(1/scale) and only divides where that could
 // change the rounded integer: with |x/scale| <= 127 (1 + 2^-23), the product
-// x*r differs from the exact quotient by less than 127 * 2^-22.9 and
-// fl32(x/scale) differs from it by at most 127 * 2^-24, so the two round to
-// the same integer unless x*r lies within 2^-15 of a half-integer; there the
-// kernel computes the IEEE quotient (__fdiv_rn) and rounds that.  Rows whose
-// reciprocal is not a finite normal number (scale below 2^-126) take the
-// division for every element.
+// x*r differs from the exact quotient by less than 2^-16 and fl32(x/scale)
+// differs from it by at most 2^-18, so both round to the same integer unless
+// x*r lies within 2^-15 of a half-integer; a vector holding such an element
+// is redone with IEEE division (__fdiv_rn) in an out-of-line path.  Rows
+// whose scale is not a normal number, or whose reciprocal is not finite,
+// take the division for every element.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -33,14 +35,6 @@
 
 namespace w8a8 {
 namespace {
-
-__device__ __forceinline__ uint4 ld_stream_16B(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
 
 template <typename T>
 struct Vec;
@@ -81,47 +75,62 @@ __device__ __forceinline__ float vec_absmax(const uint4& v) {
   return m;
 }
 
-// One code, decided as rne(fl32(x / s)) clamped to +-127 (see file header).
-__device__ __forceinline__ int quantize_one(float x, float s, float r, bool fast) {
-  float t;
-  if (fast) {
-    t = __fmul_rn(x, r);
-    const float d = fabsf(t - floorf(t) - 0.5f);
-    if (d <= 3.0517578125e-05f) t = __fdiv_rn(x, s);  // within 2^-15 of a tie
-  } else {
-    t = __fdiv_rn(x, s);
-  }
-  int q = __float2int_rn(t);
-  q = q > 127 ? 127 : q;
-  q = q < -127 ? -127 : q;
-  return q;
+__device__ __forceinline__ int clamp127(int q) { return max(-127, min(127, q)); }
+
+template <int E>
+__device__ __forceinline__ uint32_t pack4(const int (&q)[E], int w) {
+  return (static_cast<uint32_t>(q[4 * w]) & 0xFFu) | ((static_cast<uint32_t>(q[4 * w + 1]) & 0xFFu) << 8) |
+         ((static_cast<uint32_t>(q[4 * w + 2]) & 0xFFu) << 16) | (static_cast<uint32_t>(q[4 * w + 3]) << 24);
 }
 
+template <int E>
+__device__ __forceinline__ void store_codes(const int (&q)[E], int8_t* dst) {
+  if constexpr (E == 8) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack4<E>(q, 0), pack4<E>(q, 1));
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pack4<E>(q, 0);
+  }
+}
+
+// The exact path: every element as rne(fl32(x / s)) clamped to +-127.
 template <typename T>
-__device__ __forceinline__ void quantize_vec(const uint4& v, float s, float r, bool fast, bool zero,
-                                             int8_t* dst) {
+__device__ __noinline__ void quantize_vec_div(uint4 v, float s, int8_t* dst) {
   constexpr int E = Vec<T>::kElems;
   float f[E];
   Vec<T>::unpack(v, f);
-  uint32_t packed[E / 4];
+  int q[E];
 #pragma unroll
-  for (int w = 0; w < E / 4; ++w) {
-    uint32_t word = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int q = zero ? 0 : quantize_one(f[4 * w + i], s, r, fast);
-      word |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * i);
-    }
-    packed[w] = word;
-  }
-  if constexpr (E == 8) {
-    *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-  } else {
-    *reinterpret_cast<uint32_t*>(dst) = packed[0];
-  }
+  for (int i = 0; i < E; ++i) q[i] = clamp127(__float2int_rn(__fdiv_rn(f[i], s)));
+  store_codes<E>(q, dst);
 }
 
-template <typename T, int VPL>
+// The product path with the tie check described in the file header.
+template <typename T>
+__device__ __forceinline__ void quantize_vec(const uint4& v, float s, float r, bool fast, int8_t* dst) {
+  constexpr int E = Vec<T>::kElems;
+  if (!fast) {
+    quantize_vec_div<T>(v, s, dst);
+    return;
+  }
+  float f[E];
+  Vec<T>::unpack(v, f);
+  int q[E];
+  bool near_tie = false;
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    const float t = __fmul_rn(f[i], r);
+    const float n = rintf(t);
+    near_tie |= fabsf(t - n) >= 0.499969482421875f;  // 0.5 - 2^-15
+    q[i] = clamp127(__float2int_rn(n));
+  }
+  if (near_tie) {
+    quantize_vec_div<T>(v, s, dst);
+    return;
+  }
+  store_codes<E>(q, dst);
+}
+
+template <typename T>
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict__ x, int64_t M, int64_t K,
                                                             int64_t ldx, int8_t* __restrict__ q, int64_t ldq,
                                                             float* __restrict__ scale) {
@@ -130,60 +139,53 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict_
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= M) return;
 
-  const char* xr = reinterpret_cast<const char*>(x + row * ldx);
+  const uint4* xr = reinterpret_cast<const uint4*>(x + row * ldx);
   int8_t* qr = q + row * ldq;
-  const int64_t nvec = K / E;
+  const int nvec = static_cast<int>(K / E);
 
-  uint4 cache[VPL];
+  // pass 1: absmax, four 16-byte loads per lane in flight
   float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    const int64_t v = lane + 32 * i;
-    if (v < nvec) {
-      cache[i] = ld_stream_16B(xr + 16 * v);
-      amax = fmaxf(amax, vec_absmax<T>(cache[i]));
-    }
+  int v = lane;
+  for (; v + 96 < nvec; v += 128) {
+    const uint4 a0 = __ldg(xr + v), a1 = __ldg(xr + v + 32), a2 = __ldg(xr + v + 64), a3 = __ldg(xr + v + 96);
+    amax = fmaxf(amax, fmaxf(fmaxf(vec_absmax<T>(a0), vec_absmax<T>(a1)),
+                             fmaxf(vec_absmax<T>(a2), vec_absmax<T>(a3))));
   }
-  for (int64_t v = lane + 32 * VPL; v < nvec; v += 32) {
-    amax = fmaxf(amax, vec_absmax<T>(__ldg(reinterpret_cast<const uint4*>(xr) + v)));
-  }
+  for (; v < nvec; v += 32) amax = fmaxf(amax, vec_absmax<T>(__ldg(xr + v)));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
 
   const float s = __fdiv_rn(amax, 127.0f);
-  const bool zero = (s == 0.0f);
-  const float r = zero ? 0.0f : __frcp_rn(s);
-  // The product shortcut needs a normal scale and a finite reciprocal.
-  const bool fast = !zero && s >= 1.17549435e-38f && isfinite(r);
   if (lane == 0) scale[row] = s;
+  if (s == 0.0f) {  // all-zero row (or an fp32 row whose scale underflows): all codes 0
+    for (v = lane; v < nvec; v += 32) {
+      if constexpr (E == 8) {
+        *reinterpret_cast<uint2*>(qr + E * v) = make_uint2(0u, 0u);
+      } else {
+        *reinterpret_cast<uint32_t*>(qr + E * v) = 0u;
+      }
+    }
+    return;
+  }
+  const float r = __frcp_rn(s);
+  const bool fast = s >= 1.17549435e-38f && isfinite(r);
 
-#pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    const int64_t v = lane + 32 * i;
-    if (v < nvec) quantize_vec<T>(cache[i], s, r, fast, zero, qr + E * v);
+  // pass 2: codes (the row is read again, from L1)
+  v = lane;
+  for (; v + 32 < nvec; v += 64) {
+    const uint4 a0 = __ldg(xr + v), a1 = __ldg(xr + v + 32);
+    quantize_vec<T>(a0, s, r, fast, qr + E * v);
+    quantize_vec<T>(a1, s, r, fast, qr + E * (v + 32));
   }
-  for (int64_t v = lane + 32 * VPL; v < nvec; v += 32) {
-    quantize_vec<T>(__ldg(reinterpret_cast<const uint4*>(xr) + v), s, r, fast, zero, qr + E * v);
-  }
+  for (; v < nvec; v += 32) quantize_vec<T>(__ldg(xr + v), s, r, fast, qr + E * v);
 }
 
 template <typename T>
 cudaError_t launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq, float* scale,
                             cudaStream_t stream) {
-  constexpr int E = Vec<T>::kElems;
-  const int64_t per_lane = (K / E + 31) / 32;
   const int threads = 256;
   const int64_t blocks = (M + (threads / 32) - 1) / (threads / 32);
-  const dim3 grid(static_cast<unsigned>(blocks));
-  if (per_lane <= 4) {
-    quantize_rows_kernel<T, 4><<<grid, threads, 0, stream>>>(x, M, K, ldx, q, ldq, scale);
-  } else if (per_lane <= 8) {
-    quantize_rows_kernel<T, 8><<<grid, threads, 0, stream>>>(x, M, K, ldx, q, ldq, scale);
-  } else if (per_lane <= 12) {
-    quantize_rows_kernel<T, 12><<<grid, threads, 0, stream>>>(x, M, K, ldx, q, ldq, scale);
-  } else {
-    quantize_rows_kernel<T, 16><<<grid, threads, 0, stream>>>(x, M, K, ldx, q, ldq, scale);
-  }
+  quantize_rows_kernel<T><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, M, K, ldx, q, ldq, scale);
   return cudaGetLastError();
 }
 
