@@ -71,15 +71,17 @@ w8a8_status check_config(const w8a8_gemm_config& c) {
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Per-shape choice of the output tile (the paper autotunes its kernel per
-// GEMM shape).  Candidates: 256 x 256 and 256 x 128 tiles computed by CTA
-// pairs (cta_group::2; each SM stages half of B, so more ring stages fit and
-// less operand traffic flows per multiply-add), and 128 x 256 / 128 x 128
-// tiles on single CTAs for short M.  Each persistent CTA (pair) does
-// ceil(tiles / units) tiles; a tile costs its area times (K blocks + a
-// fixed per-tile overhead), scaled by the shape's relative efficiency.
+// GEMM shape; here a cost model over measured per-tile efficiencies).
+// Candidates: 128 x 256 tiles on single CTAs, 256 x 256 tiles on CTA pairs
+// (cta_group::2), and the narrower 128 x 128 / 256 x 128 tiles, which keep
+// more CTAs busy on small problems but need about twice the operand bytes
+// per multiply-add and measured ~1.7-1.9x slower per operation on B200.
+// Each persistent CTA (pair) does ceil(tiles / units) tiles; a tile costs
+// its multiply-adds times its relative cost, plus a fixed fill / drain
+// overhead of two K blocks.
 w8a8_gemm_config select(int64_t M, int64_t N, int64_t K, int sms) {
-  struct Cand { int bm, bn; double rel_cost; };
-  const Cand cands[4] = {{256, 256, 1.00}, {256, 128, 1.08}, {128, 256, 1.30}, {128, 128, 1.45}};
+  struct Cand { int bm, bn; double rel_cost; int raster; };
+  const Cand cands[4] = {{128, 256, 1.00, 1}, {256, 256, 1.02, 8}, {128, 128, 1.75, 1}, {256, 128, 1.90, 8}};
   double best = 1e300;
   w8a8_gemm_config cfg{};
   const double kblocks = static_cast<double>(ceil_div(K, 128));
@@ -87,16 +89,16 @@ w8a8_gemm_config select(int64_t M, int64_t N, int64_t K, int sms) {
     const int units = c.bm == 256 ? sms / 2 : sms;
     const int64_t tiles = ceil_div(M, c.bm) * ceil_div(N, c.bn);
     const int64_t per_unit = ceil_div(tiles, units);
-    const double cost = static_cast<double>(per_unit) * c.bm * c.bn * (kblocks + 2.0) * c.rel_cost /
-                        (c.bm == 256 ? 2.0 : 1.0);
-    if (cost < best) {
+    const double macs_per_sm = static_cast<double>(c.bm / (c.bm == 256 ? 2 : 1)) * c.bn;
+    const double cost = static_cast<double>(per_unit) * macs_per_sm * (kblocks + 2.0) * c.rel_cost;
+    if (cost < best * 0.999) {
       best = cost;
       cfg.block_m = c.bm;
       cfg.block_n = c.bn;
       cfg.stages = gemm_max_stages(c.bm, c.bn);
       const int64_t used = tiles < units ? tiles : units;
       cfg.grid = static_cast<int>(used * (c.bm == 256 ? 2 : 1));
-      cfg.raster_group = 8;
+      cfg.raster_group = c.raster;
     }
   }
   return cfg;

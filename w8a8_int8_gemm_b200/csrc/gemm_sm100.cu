@@ -51,9 +51,9 @@ namespace {
 constexpr int kBlockM = 128;
 constexpr int kBlockK = 128;            // bytes of K per stage = one 128-byte swizzle row
 constexpr int kMmaK = 32;               // K per tcgen05.mma .kind::i8
-constexpr int kThreads = 192;           // 6 warps
-constexpr int kEpiWarps = 4;
-constexpr int kEpiBufBytes = 32 * 128;  // 32 rows x 128 bytes
+constexpr int kEpiWarps = 8;            // two per 32-lane quarter of tensor memory
+constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer, MMA, epilogue warps
+constexpr int kEpiBufBytes = 32 * 128;  // one staging block per epilogue warp: 32 rows x 128 bytes
 constexpr int kSmemLimit = 232448;      // dynamic shared memory per block on sm_100
 constexpr int kBarrierBytes = 256;
 
@@ -71,12 +71,17 @@ struct Params {
 
 __host__ __device__ constexpr int a_stage_bytes() { return kBlockM * kBlockK; }
 
+// Per-tile epilogue constants in shared memory: scale_w (fp32) and bias
+// (bf16) of the tile's block_n columns.
+__host__ __device__ constexpr int params_bytes(int bn) { return bn * 6; }
+
 // Dynamic shared memory of one CTA: alignment slack, the operand ring (A:
 // 128 rows, B: block_n rows, or block_n / 2 for a CTA pair), the epilogue's
-// staging buffers and the barriers.
+// staging blocks and per-tile constants, and the barriers.
 int smem_bytes(bool pair, int bn, int stages) {
   const int b_rows = pair ? bn / 2 : bn;
-  return 1024 + stages * (a_stage_bytes() + b_rows * kBlockK) + kEpiWarps * 2 * kEpiBufBytes + kBarrierBytes;
+  return 1024 + stages * (a_stage_bytes() + b_rows * kBlockK) + kEpiWarps * kEpiBufBytes + params_bytes(bn) +
+         kBarrierBytes;
 }
 
 __device__ __forceinline__ void tile_coords(int tile, const Params& p, int& mb, int& nb) {
@@ -89,51 +94,32 @@ __device__ __forceinline__ void tile_coords(int tile, const Params& p, int& mb, 
   nb = r / gsz;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat16 l = __float2bfloat16_rn(lo);
-  const __nv_bfloat16 h = __float2bfloat16_rn(hi);
-  return static_cast<uint32_t>(__bfloat16_as_ushort(l)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h)) << 16);
-}
-
-// Dequantize 32 accumulators of one row (columns n0 .. n0+31) into 16 packed
-// bf16 pairs: y = (fl32(acc) * sa) * sw[n] + bias[n], each op rounded.
-__device__ __forceinline__ void dequant_32(const uint32_t (&v)[32], float sa, int n0, const Params& p,
-                                           uint32_t* packed) {
+// Dequantize 32 accumulators of one row into 16 packed bf16 pairs:
+// y = (fl32(acc) * sa) * sw[n] + bias[n], each op rounded, with sw / bias
+// (32 columns) read from shared memory.
+__device__ __forceinline__ void dequant_32(const uint32_t (&v)[32], float sa, const float* sw_s,
+                                           const uint16_t* bias_s, uint32_t* packed) {
 #pragma unroll
   for (int g = 0; g < 4; ++g) {
-    const int n = n0 + 8 * g;
-    float sw[8], bb[8];
-    if (n < p.N) {  // N % 8 == 0: a group of 8 columns is all in or all out
-      const float4 s0 = __ldg(reinterpret_cast<const float4*>(p.scale_w + n));
-      const float4 s1 = __ldg(reinterpret_cast<const float4*>(p.scale_w + n) + 1);
-      sw[0] = s0.x; sw[1] = s0.y; sw[2] = s0.z; sw[3] = s0.w;
-      sw[4] = s1.x; sw[5] = s1.y; sw[6] = s1.z; sw[7] = s1.w;
-      if (p.bias != nullptr) {
-        const uint4 b = __ldg(reinterpret_cast<const uint4*>(p.bias + n));
-        const uint32_t w[4] = {b.x, b.y, b.z, b.w};
+    const float4 s0 = *reinterpret_cast<const float4*>(sw_s + 8 * g);
+    const float4 s1 = *reinterpret_cast<const float4*>(sw_s + 8 * g + 4);
+    const uint4 bw = *reinterpret_cast<const uint4*>(bias_s + 8 * g);
+    const float sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    const uint32_t w[4] = {bw.x, bw.y, bw.z, bw.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          bb[2 * i] = __uint_as_float(w[i] << 16);
-          bb[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-        }
-      } else {
+    for (int i = 0; i < 4; ++i) {
+      float y[2];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) bb[i] = 0.0f;
+      for (int j = 0; j < 2; ++j) {
+        const float b = __uint_as_float(j ? (w[i] & 0xFFFF0000u) : (w[i] << 16));
+        float t = __int2float_rn(static_cast<int>(v[8 * g + 2 * i + j]));
+        t = __fmul_rn(t, sa);
+        t = __fmul_rn(t, sw[2 * i + j]);
+        y[j] = __fadd_rn(t, b);
       }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) { sw[i] = 0.0f; bb[i] = 0.0f; }
+      const __nv_bfloat162 h = __floats2bfloat162_rn(y[0], y[1]);
+      packed[4 * g + i] = *reinterpret_cast<const uint32_t*>(&h);
     }
-    float y[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float t = __int2float_rn(static_cast<int>(v[8 * g + i]));
-      t = __fmul_rn(t, sa);
-      t = __fmul_rn(t, sw[i]);
-      y[i] = __fadd_rn(t, bb[i]);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) packed[4 * g + i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
   }
 }
 
@@ -156,7 +142,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kB = kBRows * kBlockK;
   constexpr uint32_t kTxBytes = (PAIR ? 2 : 1) * (kA + kB);
   constexpr uint32_t kTmemCols = 2 * BN;  // two accumulator buffers; 256 or 512 (power of two)
-  constexpr int kColsPerChunk = (OUT == GemmOut::kBf16Dequant) ? 64 : 32;  // 128 output bytes per row
   constexpr uint32_t kIdesc = make_idesc_i8(kTileM, BN);
   constexpr int kEpiArrivals = (PAIR ? 2 : 1) * kEpiWarps;
 
@@ -166,7 +151,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sA = smem;
   uint8_t* sB = sA + stages * kA;
   uint8_t* sEpi = sB + stages * kB;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + kEpiWarps * 2 * kEpiBufBytes);
+  float* ps_w = reinterpret_cast<float*>(sEpi + kEpiWarps * kEpiBufBytes);
+  uint16_t* ps_b = reinterpret_cast<uint16_t*>(ps_w + BN);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + kEpiWarps * kEpiBufBytes + params_bytes(BN));
   uint64_t* empty = full + stages;
   uint64_t* tfull = empty + stages;
   uint64_t* tempty = tfull + 2;
@@ -224,6 +211,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t phase = 0;
     int64_t fills = 0;
     bool ok = true;
+    // Both operands are read again by other tiles: keep them in L2 ahead of
+    // the streamed output.
+    const uint64_t keep = l2_policy_evict_last();
     for (int tile = unit; ok && tile < p.num_tiles; tile += num_units) {
       int mb, nb;
       tile_coords(tile, p, mb, nb);
@@ -236,12 +226,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (PAIR) {
             const uint32_t bar = map_to_cta(smem_u32(&full[stage]), 0u);
             if (leader) mbar_arrive_expect_tx(&full[stage], kTxBytes);
-            tma_load_2d_pair(sA + stage * kA, &tm_a, bar, kb * kBlockK, a_row);
-            tma_load_2d_pair(sB + stage * kB, &tm_b, bar, kb * kBlockK, b_row);
+            tma_load_2d_pair_hint(sA + stage * kA, &tm_a, bar, kb * kBlockK, a_row, keep);
+            tma_load_2d_pair_hint(sB + stage * kB, &tm_b, bar, kb * kBlockK, b_row, keep);
           } else {
             mbar_arrive_expect_tx(&full[stage], kTxBytes);
-            tma_load_2d(sA + stage * kA, &tm_a, &full[stage], kb * kBlockK, a_row);
-            tma_load_2d(sB + stage * kB, &tm_b, &full[stage], kb * kBlockK, b_row);
+            tma_load_2d_hint(sA + stage * kA, &tm_a, &full[stage], kb * kBlockK, a_row, keep);
+            tma_load_2d_hint(sB + stage * kB, &tm_b, &full[stage], kb * kBlockK, b_row, keep);
           }
         }
         __syncwarp();
@@ -334,11 +324,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // --------------------------------------------------------- epilogue
-    const int quarter = warp & 3;  // tensor-memory lanes 32*quarter .. +31
-    const int ew = warp - 2;
-    uint8_t* bufs[2] = {sEpi + (2 * ew) * kEpiBufBytes, sEpi + (2 * ew + 1) * kEpiBufBytes};
+    // Warp e = warp - 2 reads tensor-memory lanes 32 * (warp % 4) .. +31 (the
+    // quarter a warp may address) and columns half * BN/2 .. +BN/2 of the
+    // accumulator, 32 columns at a time, loading the next 32 while it
+    // converts the current ones.
+    constexpr int kSub = BN / 2 / 32;                                       // 32-column loads per tile
+    constexpr int kSubPerStore = (OUT == GemmOut::kBf16Dequant) ? 2 : 1;    // loads per 128-byte row block
+    const int e = warp - 2;
+    const int quarter = warp & 3;
+    const int half = e >> 2;
+    uint8_t* sbuf = sEpi + e * kEpiBufBytes;
+    const uint64_t stream_out = l2_policy_evict_first();  // the output is not read again here
     int local = 0;
-    int nstores = 0;
     bool ok = true;
     for (int tile = unit; ok && tile < p.num_tiles; tile += num_units, ++local) {
       int mb, nb;
@@ -354,29 +351,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       float sa = 0.0f;
       if constexpr (OUT == GemmOut::kBf16Dequant) {
         if (row < p.M) sa = __ldg(p.scale_a + row);
-      }
-      const uint32_t t_row =
-          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * BN);
-
-#pragma unroll 1
-      for (int c = 0; c < BN / kColsPerChunk; ++c) {
-        const int col0 = nb * BN + c * kColsPerChunk;
-        uint32_t packed[32];
-        if constexpr (OUT == GemmOut::kBf16Dequant) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t v[32];
-            tmem_load_32cols(t_row + c * 64 + h * 32, v);
-            dequant_32(v, sa, col0 + h * 32, p, packed + 16 * h);
-          }
-        } else {
-          uint32_t v[32];
-          tmem_load_32cols(t_row + c * 32, v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) packed[i] = v[i];
+        // This tile's scale_w and bias, staged once for all epilogue warps
+        // (the first barrier: every warp is done with the previous tile's).
+        named_barrier_sync(1, 32 * kEpiWarps);
+        for (int i = e * 32 + lane; i < BN; i += 32 * kEpiWarps) {
+          const int n = nb * BN + i;
+          ps_w[i] = n < p.N ? __ldg(p.scale_w + n) : 0.0f;
+          ps_b[i] = (n < p.N && p.bias != nullptr) ? __bfloat16_as_ushort(p.bias[n]) : static_cast<uint16_t>(0);
         }
-        if (c == BN / kColsPerChunk - 1) {
-          // All of this warp's reads of the accumulator buffer are done.
+        named_barrier_sync(1, 32 * kEpiWarps);
+      }
+      const uint32_t t_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                              static_cast<uint32_t>(buf * BN + half * (BN / 2));
+
+      uint32_t va[32], vb[32];
+      tmem_load_32cols_async(t_base, va);
+      tmem_wait_load(va);
+#pragma unroll
+      for (int sc = 0; sc < kSub; ++sc) {
+        uint32_t(&cur)[32] = (sc & 1) ? vb : va;
+        uint32_t(&nxt)[32] = (sc & 1) ? va : vb;
+        if (sc + 1 < kSub) tmem_load_32cols_async(t_base + 32 * (sc + 1), nxt);
+        if (sc + 1 == kSub) {
+          // The last load of this accumulator buffer has completed.
           tc_fence_before_sync();
           __syncwarp();
           if (lane == 0) {
@@ -387,25 +384,46 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (row0 >= p.M || col0 >= p.N) continue;  // block entirely outside the output
-        uint8_t* sb = bufs[nstores & 1];
-        // The store that last read this staging buffer must have finished reading it.
-        if (lane == 0) bulk_wait_group_read<1>();
-        __syncwarp();
+        const int cl = half * (BN / 2) + 32 * sc;  // column inside the tile
+        const int col0 = nb * BN + cl - 32 * (sc % kSubPerStore);  // first column of the 128-byte block
+        const bool in_range = row0 < p.M && col0 < p.N;
+        if (in_range && sc % kSubPerStore == 0) {
+          // The previous store from this block must have finished reading it.
+          if (lane == 0) bulk_wait_group_read<0>();
+          __syncwarp();
+        }
+        if constexpr (OUT == GemmOut::kBf16Dequant) {
+          uint32_t pk[16];
+          dequant_32(cur, sa, ps_w + cl, ps_b + cl, pk);
+          if (in_range) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int pos = j ^ (lane & 7);  // 128-byte swizzle: 16-byte chunk j of row `lane`
-          *reinterpret_cast<uint4*>(sb + lane * 128 + pos * 16) =
-              make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+            for (int j = 0; j < 4; ++j) {
+              const int chunk = 4 * (sc % 2) + j;  // 16-byte chunk of the 128-byte row
+              const int pos = chunk ^ (lane & 7);  // 128-byte swizzle
+              *reinterpret_cast<uint4*>(sbuf + lane * 128 + pos * 16) =
+                  make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            }
+          }
+        } else {
+          if (in_range) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int pos = j ^ (lane & 7);
+              *reinterpret_cast<uint4*>(sbuf + lane * 128 + pos * 16) =
+                  make_uint4(cur[4 * j], cur[4 * j + 1], cur[4 * j + 2], cur[4 * j + 3]);
+            }
+          }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tm_d, sb, col0, row0);
-          bulk_commit_group();
+        if (in_range && (sc + 1) % kSubPerStore == 0) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tm_d, sbuf, col0, row0);
+            bulk_commit_group();
+          }
+          __syncwarp();
         }
-        __syncwarp();
-        ++nstores;
+        if (sc + 1 < kSub) tmem_wait_load(nxt);
       }
     }
     if (!ok && PAIR && lane == 0) st_cluster_u32(peer_abort, 1u);
