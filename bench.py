@@ -54,7 +54,7 @@ SPEC_INT8_POPS = 4500.0          # B200 dense int8, TOPS
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 GEMM_SOURCES = ["w8a8_int8_gemm_b200/csrc/gemm_sm100.cu", "w8a8_int8_gemm_b200/csrc/sm100_ptx.cuh",
-                "w8a8_int8_gemm_b200/csrc/api.cu"]
+                "w8a8_int8_gemm_b200/csrc/quant_row.cuh", "w8a8_int8_gemm_b200/csrc/api.cu"]
 
 
 # ---------------------------------------------------------------- helpers
@@ -86,10 +86,10 @@ def gemm_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload: str) -> dict | None:
-    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
-    taken on the current GEMM sources (else None)."""
-    path = os.path.join(ROOT, "profiles", f"gemm_{workload}_dram.json")
+def ncu_traffic(workload: str, path_kind: str) -> dict | None:
+    """DRAM bytes per launch of the step's dominant kernel from the committed
+    ncu summary, if it was taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", f"dram_{path_kind}_{workload}.json")
     try:
         with open(path) as fh:
             d = json.load(fh)
@@ -249,8 +249,16 @@ def run_native(args, wl) -> None:
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
-    stream = torch.cuda.current_stream(dev)
+    # One dedicated stream (graph capture cannot use the legacy default stream).
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        _run_native_on(args, wl, w8, rank, world, local, dev, stream)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
 
+
+def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
     # seeded inputs; each rank has its own token batch, the weight is replicated
     M, N, K = wl.M, wl.N, wl.K
     if wl.kind != "linear":
@@ -264,24 +272,35 @@ def run_native(args, wl) -> None:
 
     set_bytes = M * K * 2 + N * K + M * K + M * N * 2 + 4 * M
     nsets = max(2, int(np.ceil(3 * L2_BYTES / set_bytes)))
+    sync_words = w8.w8a8_linear_sync_words(M)
     sets = []
     for i in range(nsets):
         x = x_host.to(dev) if i == 0 else torch.roll(sets[0]["x"], shifts=i, dims=0)
         sets.append({"x": x.contiguous(), "wq": wq0 if i == 0 else wq0.clone(),
                      "xq": torch.empty((M, K), dtype=torch.int8, device=dev),
                      "sa": torch.empty((M,), dtype=torch.float32, device=dev),
+                     "sync": torch.zeros((sync_words,), dtype=torch.int32, device=dev),
                      "out": torch.empty((M, N), dtype=torch.bfloat16, device=dev)})
 
-    def step(i, evs=None):
+    def step_fused(i):
         s = sets[i % nsets]
-        if evs is not None:
-            evs[0].record(stream)
+        w8.w8a8_linear_fused(s["x"], s["wq"], sw, bias, out=s["out"], ws_xq=s["xq"], ws_scale_a=s["sa"],
+                             ws_sync=s["sync"], stream=stream)
+
+    def step_linear(i):
+        s = sets[i % nsets]
+        w8.w8a8_linear(s["x"], s["wq"], sw, bias, out=s["out"], ws_xq=s["xq"], ws_scale_a=s["sa"], stream=stream)
+
+    def step_quant(i):
+        s = sets[i % nsets]
         w8.w8a8_quantize_act(s["x"], xq=s["xq"], scale_a=s["sa"], stream=stream)
-        if evs is not None:
-            evs[1].record(stream)
+
+    def step_gemm(i):
+        s = sets[i % nsets]
         w8.w8a8_gemm(s["xq"], s["wq"], s["sa"], sw, bias, out=s["out"], stream=stream)
-        if evs is not None:
-            evs[2].record(stream)
+
+    step = step_fused if args.path == "fused" else step_linear
+    launches_per_step = 1 if args.path == "fused" else 2
 
     for i in range(args.warmup):
         step(i)
@@ -289,8 +308,23 @@ def run_native(args, wl) -> None:
     if w8.w8a8_read_device_error() != 0:
         raise SystemExit("a kernel wait timed out during warm-up")
 
-    # timed region
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    def capture(fn, n):
+        """A CUDA graph of n back-to-back calls of fn (cycling the buffer sets)."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+            for i in range(n):
+                fn(i)
+        return g
+
+    # The timed region replays CUDA graphs of the step (the host launch cost of
+    # the Python binding is not part of the layer); exactly K steps run.
+    G = nsets * max(1, 32 // nsets)
+    g_main = capture(step, G)
+    g_tail = capture(step, args.steps % G) if args.steps % G else None
+    n_main = args.steps // G
+    g_main.replay()
+    torch.cuda.synchronize(dev)
+
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -299,8 +333,10 @@ def run_native(args, wl) -> None:
     sampler = ClockSampler(local)
     time.sleep(0.3)
     start.record(stream)
-    for i in range(args.steps):
-        step(i, evs[i])
+    for _ in range(n_main):
+        g_main.replay()
+    if g_tail is not None:
+        g_tail.replay()
     end.record(stream)
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
@@ -315,20 +351,44 @@ def run_native(args, wl) -> None:
     if code != 0:
         raise SystemExit(f"a kernel wait timed out in the timed region (site {code})")
 
-    q_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    g_ms = [e[1].elapsed_time(e[2]) for e in evs]
     ms_step = elapsed_ms / args.steps
     ops = 2.0 * M * N * K
     value = ops * world / (ms_step * 1e-3) / 1e12
 
+    def graph_ms(fn, reps):
+        """Mean ms per call of fn: a graph of G calls, timed with CUDA events."""
+        try:
+            g = capture(fn, G)
+        except RuntimeError as exc:  # e.g. a launch kind the graph cannot hold
+            print(f"[bench] could not capture {fn.__name__}: {exc}", file=sys.stderr)
+            torch.cuda.synchronize(dev)
+            return None
+        g.replay()
+        a_ev = torch.cuda.Event(enable_timing=True)
+        b_ev = torch.cuda.Event(enable_timing=True)
+        a_ev.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b_ev.record(stream)
+        torch.cuda.synchronize(dev)
+        return a_ev.elapsed_time(b_ev) / (reps * G)
+
     peaks = measured_peaks()
-    gemm_ms = statistics.fmean(g_ms)
-    quant_ms = statistics.fmean(q_ms)
     int8_peak = peaks["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
-    gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
     quant_bytes = 3 * M * K + 4 * M
-    quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
-    traffic = ncu_traffic(wl.name)
+    # The dominant kernel on its own: the GEMM (both paths spend ~90% of the
+    # step in it), timed the same way on the same buffer sets.
+    kernel_fn = step_fused if args.path == "fused" else step_gemm
+    kernel_ms = graph_ms(kernel_fn, max(3, 300 // G))
+    kernel_tops = ops / (kernel_ms * 1e-3) / 1e12
+    side = {}
+    if rank == 0 and not args.no_context:
+        side["quant_ms"] = graph_ms(step_quant, max(3, 300 // G))
+        side["gemm_ms"] = kernel_ms if args.path != "fused" else graph_ms(step_gemm, max(3, 300 // G))
+        side["linear_ms"] = graph_ms(step_linear, max(3, 300 // G))
+        side["fused_ms"] = graph_ms(step_fused, max(3, 300 // G))
+        side = {k: v for k, v in side.items() if v is not None}
+    traffic = ncu_traffic(wl.name, args.path)
 
     result = None
     if rank == 0:
@@ -336,32 +396,48 @@ def run_native(args, wl) -> None:
         ctx = context_baselines(wl, d, sets[0], sw, bias, dev, args) if not args.no_context else None
         cpu = cpu_baseline(wl) if (world == 1 and not args.no_cpu_baseline) else None
         cfg = wl_config(wl)
+        cfg["path"] = ("one fused kernel per step (w8a8_linear_fused)" if args.path == "fused"
+                       else "w8a8_linear per step: quantizer kernel, then the GEMM kernel as its "
+                            "programmatic dependent")
+        cfg["timing"] = f"CUDA graphs of {G} steps replayed; events around the whole timed region"
         cfg["parallelism"] = f"dp{world} (independent token batches, replicated weight)"
         cfg["gemm_config"] = w8.w8a8_select_config(M, N, K)
         cfg["buffer_sets"] = nsets
         cfg["footprint_mb"] = round(nsets * set_bytes / 2 ** 20, 1)
+        kname = ("gemm_w8a8_kernel, fused (quantize + GEMM + epilogue)" if args.path == "fused"
+                 else "gemm_w8a8_kernel (GEMM + dequant/bias epilogue)")
         result = {
             "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded; stands in for Ideogram 4.0 "
             "DiT activations and weights, which are not available)", "config": cfg,
-            "roofline": {"bound": "tensor", "achieved": gemm_tops, "peak": int8_peak, "unit": "TOPS",
-                         "frac": gemm_tops / int8_peak,
+            "roofline": {"bound": "tensor", "achieved": kernel_tops, "peak": int8_peak, "unit": "TOPS",
+                         "frac": kernel_tops / int8_peak,
                          "traffic": traffic["dram_bytes_per_launch"] if traffic else None,
-                         "kernel": "gemm_w8a8_kernel",
+                         "kernel": kname, "ms_per_launch": kernel_ms,
+                         "timing": "CUDA events around graph replays of back-to-back launches of this kernel "
+                                   "on the benchmark's rotating buffer sets, right after the timed region",
                          "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x "
-                                        f"{NOMINAL_INT8_OVER_BF16} (nominal int8/bf16 ratio)"},
-            "gemm": {"ms": gemm_ms, "tops": gemm_tops, "pct_of_spec_4p5_pops": 100 * gemm_tops / SPEC_INT8_POPS,
-                     "algorithmic_bytes": M * K + N * K + 2 * M * N + 4 * M + 4 * N + 2 * N},
-            "quantizer": {"ms": quant_ms, "gbs": quant_gbs, "frac_of_measured_hbm": quant_gbs / peaks["hbm_gbs"],
-                          "frac_of_8tbs": quant_gbs / 8000.0, "bytes": quant_bytes},
-            "e2e": e2e, "gpu_launches": 2 * args.steps, "clocks": clocks,
+                                        f"{NOMINAL_INT8_OVER_BF16} (nominal dense int8/bf16 ratio)"},
+            "pct_of_spec_int8_4p5_pops": 100 * kernel_tops / SPEC_INT8_POPS,
+            "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
             "cpu_baseline": cpu, "context": ctx,
         }
+        if side:
+            result["components"] = {
+                "note": "after the timed region: graphs of back-to-back calls of one entry point",
+            }
+            if "quant_ms" in side:
+                qg = quant_bytes / (side["quant_ms"] * 1e-3) / 1e9
+                result["components"]["quantizer"] = {"ms": side["quant_ms"], "gbs": qg,
+                                                     "frac_of_measured_hbm": qg / peaks["hbm_gbs"],
+                                                     "frac_of_8tbs": qg / 8000.0, "bytes": quant_bytes}
+            for key, name in (("gemm_ms", "gemm"), ("linear_ms", "w8a8_linear"), ("fused_ms", "w8a8_linear_fused")):
+                if key in side:
+                    tops = ops / (side[key] * 1e-3) / 1e12
+                    result["components"][name] = {"ms": side[key], "tops": tops,
+                                                  "pct_of_spec_int8_4p5_pops": 100 * tops / SPEC_INT8_POPS}
         print(json.dumps(result), flush=True)
-    if world > 1:
-        torch.distributed.barrier()
-        torch.distributed.destroy_process_group()
 
 
 def run_e2e(w8, wl, x_host, wq, sw, bias, dev, stream, args) -> dict:
@@ -374,10 +450,14 @@ def run_e2e(w8, wl, x_host, wq, sw, bias, dev, stream, args) -> dict:
     od = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     xq = torch.empty((M, K), dtype=torch.int8, device=dev)
     sa = torch.empty((M,), dtype=torch.float32, device=dev)
+    sync = torch.zeros((w8.w8a8_linear_sync_words(M),), dtype=torch.int32, device=dev)
 
     def one():
         xd.copy_(xh, non_blocking=True)
-        w8.w8a8_linear(xd, wq, sw, bias, out=od, ws_xq=xq, ws_scale_a=sa, stream=stream)
+        if args.path == "fused":
+            w8.w8a8_linear_fused(xd, wq, sw, bias, out=od, ws_xq=xq, ws_scale_a=sa, ws_sync=sync, stream=stream)
+        else:
+            w8.w8a8_linear(xd, wq, sw, bias, out=od, ws_xq=xq, ws_scale_a=sa, stream=stream)
         oh.copy_(od, non_blocking=True)
 
     for _ in range(3):
@@ -438,11 +518,13 @@ def context_baselines(wl, d, s0, sw, bias, dev, args) -> dict:
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=6000)
+    ap.add_argument("--steps", type=int, default=12000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--path", default="two-kernel", choices=["fused", "two-kernel"],
+                    help="w8a8_linear (quantizer + GEMM, default) or the one-kernel w8a8_linear_fused")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-context", action="store_true")
     args = ap.parse_args(argv)

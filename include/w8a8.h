@@ -132,6 +132,30 @@ W8A8_API w8a8_status w8a8_linear(const void* x, const int8_t* wq, const float* s
                         int64_t M, int64_t N, int64_t K, w8a8_stream_t stream);
 
 /*
+ * The same layer as ONE kernel (the paper's "single fused" kernel, abstract,
+ * extended to the quantizer): the GEMM kernel's epilogue warps quantize the
+ * activation rows into the workspace first, and the tensor-core pipeline
+ * starts on each 128-row block as soon as that block is quantized, so the
+ * quantizer's memory traffic overlaps the GEMM instead of preceding it.
+ *   Arguments as in w8a8_linear, plus
+ *   ws_sync  uint32 [w8a8_linear_sync_words(M)]: row-block counters.  The
+ *            caller zeroes it ONCE (e.g. cudaMemset) before the first call;
+ *            every call that completes leaves it zeroed again.  After a call
+ *            that reported W8A8_ERR_TIMEOUT it must be zeroed again.
+ * Calls sharing one ws_sync (or one ws_xq / ws_scale_a) must not overlap on
+ * the GPU.  Needs every CTA of the grid resident at once (a cooperative
+ * launch); if the device cannot guarantee that, the call fails with
+ * W8A8_ERR_LAUNCH and nothing runs.  Results are bit-identical to
+ * w8a8_linear.
+ */
+W8A8_API w8a8_status w8a8_linear_fused(const void* x, const int8_t* wq, const float* scale_w, const void* bias,
+                                       void* out, int8_t* ws_xq, float* ws_scale_a, uint32_t* ws_sync,
+                                       int64_t M, int64_t N, int64_t K, w8a8_stream_t stream);
+
+/* Number of uint32 words of ws_sync for M tokens (M >= 0): ceil(M/128) + 1. */
+W8A8_API int64_t w8a8_linear_sync_words(int64_t M);
+
+/*
  * The GEMM without the epilogue: raw int32 accumulators
  *   acc[m,n] = sum_k xq[m,k]*wq[n,k], acc int32 [M, N] (row stride N).
  * The abstract states the int32 accumulation is bit-exact against a library

@@ -69,6 +69,15 @@ def test_host_validation_without_device(w8):
     assert lib.w8a8_linear(A, A, A, None, A, A, A, 4, 12, 32, None) == 1
     assert lib.w8a8_linear(A, A, A, None, A, A + 1, A, 4, 8, 32, None) == 2
     assert lib.w8a8_linear(A, A, A, None, A, A, A, 0, 8, 32, None) == 0
+    # the fused layer: same checks, plus its counter workspace
+    assert lib.w8a8_linear_fused(A, A, A, None, A, A, A, None, 4, 8, 32, None) == 1   # no ws_sync
+    assert lib.w8a8_linear_fused(A, A, A, None, A, A, A, A + 4, 4, 8, 32, None) == 2  # misaligned ws_sync
+    assert lib.w8a8_linear_fused(A, A, A, None, A, A, A, A, 4, 12, 32, None) == 1     # N % 8
+    assert lib.w8a8_linear_fused(A, A, A, None, A, A, A, A, 0, 8, 32, None) == 0      # empty
+    assert lib.w8a8_linear_sync_words(0) == 1
+    assert lib.w8a8_linear_sync_words(128) == 2
+    assert lib.w8a8_linear_sync_words(129) == 3
+    assert lib.w8a8_linear_sync_words(4096) == 33
     # explicit configurations
     cfg = w8.GemmConfig(block_m=128, block_n=200, stages=4, grid=1, raster_group=1)
     assert lib.w8a8_gemm_i32_ex(A, A, A, 4, 8, 32, ctypes.byref(cfg), None) == 1

@@ -32,7 +32,20 @@ def w8():
     return mod
 
 
-def _run(w8, name, n_sample):
+ENTRY_POINTS = ["w8a8_linear", "w8a8_linear_fused"]
+
+
+def _call(w8, entry, x, wq, sw, bias, xq, sa):
+    if entry == "w8a8_linear":
+        return w8.w8a8_linear(x, wq, sw, bias, ws_xq=xq, ws_scale_a=sa)
+    sync = torch.zeros((w8.w8a8_linear_sync_words(x.shape[0]),), dtype=torch.int32, device=x.device)
+    out = w8.w8a8_linear_fused(x, wq, sw, bias, ws_xq=xq, ws_scale_a=sa, ws_sync=sync)
+    torch.cuda.synchronize()
+    assert int(sync.abs().sum()) == 0, "the fused call must leave its counters zeroed"
+    return out
+
+
+def _run(w8, name, n_sample, entry="w8a8_linear"):
     wl = workloads.WORKLOADS[name]
     d = workloads.make(wl)
     dev = torch.device("cuda")
@@ -41,7 +54,7 @@ def _run(w8, name, n_sample):
     bias = bf16_bits_to_torch(d["bias"], dev)
     xq = torch.empty((wl.M, wl.K), dtype=torch.int8, device=dev)
     sa = torch.empty((wl.M,), dtype=torch.float32, device=dev)
-    out = w8.w8a8_linear(x, wq, sw, bias, ws_xq=xq, ws_scale_a=sa)
+    out = _call(w8, entry, x, wq, sw, bias, xq, sa)
     torch.cuda.synchronize()
     assert w8.w8a8_read_device_error() == 0
 
@@ -81,22 +94,51 @@ def _run(w8, name, n_sample):
     return ulp
 
 
-def test_linear_tiny_all_rows(w8):
-    ulp = _run(w8, "tiny", None)
+@pytest.mark.parametrize("entry", ENTRY_POINTS)
+def test_linear_tiny_all_rows(w8, entry):
+    ulp = _run(w8, "tiny", None, entry)
     assert ulp.max() <= 1
 
 
+@pytest.mark.parametrize("entry", ENTRY_POINTS)
 @pytest.mark.parametrize("name", ["qkv_768", "mlp_up_1024"])
-def test_linear_dit_workloads(w8, name):
-    _run(w8, name, 40)
+def test_linear_dit_workloads(w8, name, entry):
+    _run(w8, name, 40, entry)
 
 
+@pytest.mark.parametrize("entry", ENTRY_POINTS)
 @pytest.mark.parametrize("name", ["sweep_qkv", "sweep_out", "sweep_up", "sweep_down"])
-def test_linear_block_sweep(w8, name):
-    _run(w8, name, 24)
+def test_linear_block_sweep(w8, name, entry):
+    _run(w8, name, 24, entry)
 
 
-def test_linear_ragged(w8):
+@pytest.mark.parametrize("M,N,K", [(1, 8, 16), (130, 392, 1040), (333, 520, 3088), (4096, 12288, 3072)])
+def test_fused_equals_two_kernel_path(w8, M, N, K):
+    """The fused layer gives bit-identical outputs, codes and scales, call
+    after call on the same counter workspace (which it leaves zeroed)."""
+    rng = np.random.default_rng(M + N + K)
+    dev = torch.device("cuda")
+    x = (torch.from_numpy(rng.standard_normal((M, K)).astype(np.float32)) * 3).to(torch.bfloat16).to(dev)
+    wq = torch.from_numpy(rng.integers(-127, 128, (N, K), dtype=np.int8)).to(dev)
+    sw = torch.from_numpy(np.exp(rng.uniform(-9, -3, N)).astype(np.float32)).to(dev)
+    bias = (torch.from_numpy(rng.standard_normal(N).astype(np.float32)) * 0.1).to(torch.bfloat16).to(dev)
+    xq1 = torch.empty((M, K), dtype=torch.int8, device=dev)
+    sa1 = torch.empty((M,), dtype=torch.float32, device=dev)
+    ref = w8.w8a8_linear(x, wq, sw, bias, ws_xq=xq1, ws_scale_a=sa1)
+    sync = torch.zeros((w8.w8a8_linear_sync_words(M),), dtype=torch.int32, device=dev)
+    for _ in range(3):
+        xq2 = torch.full((M, K), 7, dtype=torch.int8, device=dev)
+        sa2 = torch.full((M,), -1.0, dtype=torch.float32, device=dev)
+        out = w8.w8a8_linear_fused(x, wq, sw, bias, ws_xq=xq2, ws_scale_a=sa2, ws_sync=sync)
+        torch.cuda.synchronize()
+        assert w8.w8a8_read_device_error() == 0
+        assert int(sync.abs().sum()) == 0
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+        assert torch.equal(xq2, xq1) and torch.equal(sa2.view(torch.int32), sa1.view(torch.int32))
+
+
+@pytest.mark.parametrize("entry", ENTRY_POINTS)
+def test_linear_ragged(w8, entry):
     """Token counts that are not multiples of the tile, N not a multiple of 256."""
     rng = np.random.default_rng(5)
     dev = torch.device("cuda")
@@ -105,7 +147,9 @@ def test_linear_ragged(w8):
         w = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
         bias_bits = workloads.gen_bias(N, M)
         wq, sw = w8.w8a8_quantize_weight(torch.from_numpy(w).to(dev))
-        out = w8.w8a8_linear(bf16_bits_to_torch(x_bits, dev), wq, sw, bf16_bits_to_torch(bias_bits, dev))
+        xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+        sa = torch.empty((M,), dtype=torch.float32, device=dev)
+        out = _call(w8, entry, bf16_bits_to_torch(x_bits, dev), wq, sw, bf16_bits_to_torch(bias_bits, dev), xq, sa)
         torch.cuda.synchronize()
         wq_o, sw_o = oracle.quantize_weight(w)
         out_o, *_ = oracle.linear(x_bits, wq_o, sw_o, bias_bits)

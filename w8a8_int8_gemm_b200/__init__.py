@@ -26,7 +26,8 @@ __all__ = [
     "W8A8Error", "lib_path", "header_path", "exported_names",
     "w8a8_status_string", "w8a8_abi_version",
     "w8a8_quantize_act", "w8a8_quantize_weight", "w8a8_gemm", "w8a8_gemm_ex",
-    "w8a8_gemm_i32", "w8a8_gemm_i32_ex", "w8a8_linear", "w8a8_select_config",
+    "w8a8_gemm_i32", "w8a8_gemm_i32_ex", "w8a8_linear", "w8a8_linear_fused", "w8a8_linear_sync_words",
+    "w8a8_select_config",
     "w8a8_read_device_error", "w8a8_set_wait_timeout_ns", "w8a8_selftest_wait_timeout",
 ]
 
@@ -70,6 +71,8 @@ def _load() -> ctypes.CDLL:
         "w8a8_gemm_i32": ([p, p, p, i64, i64, i64, p], ctypes.c_int),
         "w8a8_gemm_i32_ex": ([p, p, p, i64, i64, i64, ctypes.POINTER(GemmConfig), p], ctypes.c_int),
         "w8a8_linear": ([p, p, p, p, p, p, p, i64, i64, i64, p], ctypes.c_int),
+        "w8a8_linear_fused": ([p, p, p, p, p, p, p, p, i64, i64, i64, p], ctypes.c_int),
+        "w8a8_linear_sync_words": ([i64], i64),
         "w8a8_select_config": ([i64, i64, i64, ctypes.POINTER(GemmConfig)], ctypes.c_int),
         "w8a8_read_device_error": ([ctypes.POINTER(i32), i32], ctypes.c_int),
         "w8a8_set_wait_timeout_ns": ([i64], ctypes.c_int),
@@ -285,6 +288,47 @@ def w8a8_linear(x, wq, scale_w, bias=None, out=None, ws_xq=None, ws_scale_a=None
     _need_contig(ws_scale_a, "ws_scale_a", torch.float32, (M,))
     _check(_lib.w8a8_linear(_ptr(x), _ptr(wq), _ptr(scale_w), _ptr(bias), _ptr(out), _ptr(ws_xq),
                             _ptr(ws_scale_a), M, N, K, _stream(stream, dev)), "w8a8_linear")
+    return out
+
+
+def w8a8_linear_sync_words(M: int) -> int:
+    return int(_lib.w8a8_linear_sync_words(int(M)))
+
+
+def w8a8_linear_fused(x, wq, scale_w, bias=None, out=None, ws_xq=None, ws_scale_a=None, ws_sync=None,
+                      stream=None):
+    """The W8A8 linear layer as one kernel (quantization inside the GEMM).
+
+    ws_sync: int32 tensor of w8a8_linear_sync_words(M) words, zeroed once by
+    the caller; each completed call leaves it zeroed (allocated and zeroed
+    here if not given)."""
+    _need(x, "x", torch.bfloat16, 2)
+    M, K = x.shape
+    _need(wq, "wq", torch.int8, 2)
+    N = wq.shape[0]
+    if wq.shape[1] != K:
+        raise ValueError(f"inner dimensions differ: x has K={K}, wq has K={wq.shape[1]}")
+    _need_contig(x, "x", torch.bfloat16, (M, K))
+    _need_contig(wq, "wq", torch.int8, (N, K))
+    _need_contig(scale_w, "scale_w", torch.float32, (N,))
+    if bias is not None:
+        _need_contig(bias, "bias", torch.bfloat16, (N,))
+    dev = x.device
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    if ws_xq is None:
+        ws_xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+    if ws_scale_a is None:
+        ws_scale_a = torch.empty((M,), dtype=torch.float32, device=dev)
+    if ws_sync is None:
+        ws_sync = torch.zeros((w8a8_linear_sync_words(M),), dtype=torch.int32, device=dev)
+    _need_contig(out, "out", torch.bfloat16, (M, N))
+    _need_contig(ws_xq, "ws_xq", torch.int8, (M, K))
+    _need_contig(ws_scale_a, "ws_scale_a", torch.float32, (M,))
+    _need_contig(ws_sync, "ws_sync", torch.int32, (w8a8_linear_sync_words(M),))
+    _check(_lib.w8a8_linear_fused(_ptr(x), _ptr(wq), _ptr(scale_w), _ptr(bias), _ptr(out), _ptr(ws_xq),
+                                  _ptr(ws_scale_a), _ptr(ws_sync), M, N, K, _stream(stream, dev)),
+           "w8a8_linear_fused")
     return out
 
 

@@ -22,7 +22,7 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libw8a8.so")
 
 SOURCES = ["api.cu", "quant.cu", "gemm_sm100.cu"]
-HEADERS = ["internal.h", "sm100_ptx.cuh"]
+HEADERS = ["internal.h", "sm100_ptx.cuh", "quant_row.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -79,13 +79,14 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // Each persistent CTA (pair) does ceil(tiles / units) tiles; a tile costs
 // its multiply-adds times its relative cost, plus a fixed fill / drain
 // overhead of two K blocks.
-w8a8_gemm_config select(int64_t M, int64_t N, int64_t K, int sms) {
+w8a8_gemm_config select(int64_t M, int64_t N, int64_t K, int sms, bool allow_pair = true) {
   struct Cand { int bm, bn; double rel_cost; int raster; };
   const Cand cands[4] = {{128, 256, 1.00, 1}, {256, 256, 1.02, 8}, {128, 128, 1.75, 1}, {256, 128, 1.90, 8}};
   double best = 1e300;
   w8a8_gemm_config cfg{};
   const double kblocks = static_cast<double>(ceil_div(K, 128));
   for (const Cand& c : cands) {
+    if (c.bm == 256 && !allow_pair) continue;
     const int units = c.bm == 256 ? sms / 2 : sms;
     const int64_t tiles = ceil_div(M, c.bm) * ceil_div(N, c.bn);
     const int64_t per_unit = ceil_div(tiles, units);
@@ -112,7 +113,8 @@ w8a8_status from_cuda(cudaError_t e) {
 
 w8a8_status gemm_common(const int8_t* xq, const int8_t* wq, const float* scale_a, const float* scale_w,
                         const void* bias, void* out, int64_t M, int64_t N, int64_t K,
-                        const w8a8_gemm_config* user_cfg, GemmOut kind, cudaStream_t stream) {
+                        const w8a8_gemm_config* user_cfg, GemmOut kind, cudaStream_t stream,
+                        bool overlap_prologue = false) {
   w8a8_status st = check_gemm_shape(M, N, K);
   if (st != W8A8_OK) return st;
   if (user_cfg != nullptr && (st = check_config(*user_cfg)) != W8A8_OK) return st;
@@ -138,6 +140,7 @@ w8a8_status gemm_common(const int8_t* xq, const int8_t* wq, const float* scale_a
   a.K = K;
   a.out_kind = kind;
   a.timeout_ns = static_cast<uint64_t>(g_timeout_ns.load());
+  a.overlap_prologue = overlap_prologue;
   GemmConfig c{cfg.block_m, cfg.block_n, cfg.stages, cfg.grid, cfg.raster_group};
   return from_cuda(launch_gemm(a, c, stream));
 }
@@ -233,8 +236,48 @@ w8a8_status w8a8_linear(const void* x, const int8_t* wq, const float* scale_w, c
   }
   st = w8a8_quantize_act(x, M, K, K, ws_xq, K, ws_scale_a, stream);
   if (st != W8A8_OK) return st;
-  return w8a8_gemm(ws_xq, wq, ws_scale_a, scale_w, bias, out, M, N, K, stream);
+  return gemm_common(ws_xq, wq, ws_scale_a, scale_w, bias, out, M, N, K, nullptr, GemmOut::kBf16Dequant,
+                     reinterpret_cast<cudaStream_t>(stream), /*overlap_prologue=*/true);
 }
+
+w8a8_status w8a8_linear_fused(const void* x, const int8_t* wq, const float* scale_w, const void* bias, void* out,
+                              int8_t* ws_xq, float* ws_scale_a, uint32_t* ws_sync, int64_t M, int64_t N, int64_t K,
+                              w8a8_stream_t stream) {
+  w8a8_status st = check_gemm_shape(M, N, K);
+  if (st != W8A8_OK) return st;
+  if (M == 0 || N == 0) return W8A8_OK;
+  if (x == nullptr || wq == nullptr || scale_w == nullptr || out == nullptr || ws_xq == nullptr ||
+      ws_scale_a == nullptr || ws_sync == nullptr) {
+    return W8A8_ERR_INVALID_ARG;
+  }
+  if (!aligned16(x) || !aligned16(wq) || !aligned16(scale_w) || !aligned16(bias) || !aligned16(out) ||
+      !aligned16(ws_xq) || !aligned16(ws_scale_a) || !aligned16(ws_sync)) {
+    return W8A8_ERR_ALIGNMENT;
+  }
+  DeviceInfo dev;
+  if ((st = current_device(&dev)) != W8A8_OK) return st;
+  const w8a8_gemm_config cfg = select(M, N, K, dev.sms, /*allow_pair=*/false);
+  GemmArgs a;
+  a.xq = ws_xq;
+  a.wq = wq;
+  a.scale_a = ws_scale_a;
+  a.scale_w = scale_w;
+  a.bias = bias;
+  a.out = out;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.out_kind = GemmOut::kBf16Dequant;
+  a.timeout_ns = static_cast<uint64_t>(g_timeout_ns.load());
+  a.fused = true;
+  a.x = x;
+  a.ldx = K;
+  a.sync = ws_sync;
+  GemmConfig c{cfg.block_m, cfg.block_n, cfg.stages, cfg.grid, cfg.raster_group};
+  return from_cuda(launch_gemm(a, c, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int64_t w8a8_linear_sync_words(int64_t M) { return M < 0 ? 0 : linear_sync_words(M); }
 
 w8a8_status w8a8_select_config(int64_t M, int64_t N, int64_t K, w8a8_gemm_config* cfg) {
   if (cfg == nullptr) return W8A8_ERR_INVALID_ARG;

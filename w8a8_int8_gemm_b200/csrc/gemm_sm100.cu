@@ -39,6 +39,7 @@
 #include <mutex>
 
 #include "internal.h"
+#include "quant_row.cuh"
 #include "sm100_ptx.cuh"
 
 namespace w8a8 {
@@ -67,6 +68,14 @@ struct Params {
   const __nv_bfloat16* bias;
   uint64_t timeout_ns;
   int* err;  // device error word
+  // Fused linear layer only: the bf16 activations, the workspace the kernel
+  // quantizes them into (xq is also the A operand of tm_a), and the
+  // row-block counters ([m_tiles] blocks + 1 CTA counter, zero on entry).
+  const __nv_bfloat16* x;
+  int64_t ldx;
+  int8_t* xq_out;
+  float* scale_out;
+  uint32_t* sync;
 };
 
 __host__ __device__ constexpr int a_stage_bytes() { return kBlockM * kBlockK; }
@@ -132,7 +141,16 @@ __device__ __forceinline__ void dequant_32(const uint32_t (&v)[32], float sa, co
 // stages count both CTAs' TMA bytes; the leader's commits arrive on the
 // "empty" and "accumulator full" barriers of both CTAs; both CTAs' epilogue
 // warps arrive on the leader's "accumulator empty" barrier.
-template <int BN, GemmOut OUT, bool PAIR>
+// FUSE (single CTAs only): the whole W8A8 linear layer in one kernel.  The
+// epilogue warps, idle until the first accumulator is ready, first quantize
+// the activation rows (one warp per row, rows dealt round-robin over all
+// CTAs so that low row blocks finish first) into the workspace and count
+// each finished row on its 128-row block's counter (release); the TMA
+// producer acquires a block's counter before loading that block's rows of
+// A, and the epilogue before reading its scales.  All CTAs are co-resident
+// (cooperative launch), so these waits cannot deadlock; they are bounded
+// all the same.  The last CTA to finish resets the counters to zero.
+template <int BN, GemmOut OUT, bool PAIR, bool FUSE>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_d, const Params p) {
@@ -211,6 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t phase = 0;
     int64_t fills = 0;
     bool ok = true;
+    int ready_mb = -1;  // fused layer: the last row block known to be quantized
     // Both operands are read again by other tiles: keep them in L2 ahead of
     // the streamed output.
     const uint64_t keep = l2_policy_evict_last();
@@ -226,12 +245,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (PAIR) {
             const uint32_t bar = map_to_cta(smem_u32(&full[stage]), 0u);
             if (leader) mbar_arrive_expect_tx(&full[stage], kTxBytes);
-            tma_load_2d_pair_hint(sA + stage * kA, &tm_a, bar, kb * kBlockK, a_row, keep);
             tma_load_2d_pair_hint(sB + stage * kB, &tm_b, bar, kb * kBlockK, b_row, keep);
+            if (fills == 0) pdl_wait_prerequisites();  // A may be written by the kernel before this one
+            tma_load_2d_pair_hint(sA + stage * kA, &tm_a, bar, kb * kBlockK, a_row, keep);
           } else {
             mbar_arrive_expect_tx(&full[stage], kTxBytes);
-            tma_load_2d_hint(sA + stage * kA, &tm_a, &full[stage], kb * kBlockK, a_row, keep);
             tma_load_2d_hint(sB + stage * kB, &tm_b, &full[stage], kb * kBlockK, b_row, keep);
+            if constexpr (!FUSE) {
+              if (fills == 0) pdl_wait_prerequisites();  // A may be written by the kernel before this one
+              tma_load_2d_hint(sA + stage * kA, &tm_a, &full[stage], kb * kBlockK, a_row, keep);
+            }
+          }
+        }
+        if constexpr (FUSE) {
+          if (mb != ready_mb) {
+            // This block's activation rows must be quantized before TMA reads them.
+            bool rok = true;
+            if (lane == 0) {
+              rok = counter_wait_bounded(&p.sync[mb], static_cast<uint32_t>(min(kBlockM, p.M - mb * kBlockM)),
+                                         abort_flag, p.timeout_ns, p.err, kSiteRowsReady);
+              fence_proxy_async_global();
+            }
+            ok = __shfl_sync(0xffffffffu, rok ? 1 : 0, 0) != 0;
+            if (ok) ready_mb = mb;
+          }
+          // After a failed wait the load is still issued (its data is
+          // discarded): the stage's barrier completes and teardown drains it.
+          if (lane == 0) tma_load_2d_hint(sA + stage * kA, &tm_a, &full[stage], kb * kBlockK, a_row, keep);
+          if (!ok) {
+            __syncwarp();
+            ++fills;
+            break;
           }
         }
         __syncwarp();
@@ -335,8 +379,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = e >> 2;
     uint8_t* sbuf = sEpi + e * kEpiBufBytes;
     const uint64_t stream_out = l2_policy_evict_first();  // the output is not read again here
+    if constexpr (!FUSE) pdl_wait_prerequisites();  // scale_a may come from the kernel before this one
     int local = 0;
     bool ok = true;
+    if constexpr (FUSE) {
+      // Per-token quantization of the activations.  Warp w of the grid's
+      // nq epilogue warps takes the row pairs (2w, 2w+1), (2(w+nq), ...),
+      // both rows' loads in flight together, so the low row blocks the
+      // first tiles need are finished first.
+      const int nvec = p.K / 8;
+      const int nq = static_cast<int>(gridDim.x) * kEpiWarps;
+      auto publish = [&](int r, float srow) {
+        if (lane == 0) p.scale_out[r] = srow;
+        // Publish the row: its codes are read by other CTAs' TMA (async proxy).
+        fence_proxy_async_global();
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) red_release_gpu_add(&p.sync[r / kBlockM], 1u);
+      };
+      auto xrow = [&](int r) { return reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(r) * p.ldx); };
+      auto qrow_ptr = [&](int r) { return p.xq_out + static_cast<int64_t>(r) * p.K; };
+      for (int pr = static_cast<int>(blockIdx.x) * kEpiWarps + e; 2 * pr < p.M; pr += nq) {
+        const int r = 2 * pr;
+        const int r2 = r + 1;
+        if (nvec <= 32 * 12) {
+          if (r2 < p.M) {
+            float s0, s1;
+            qrow::quantize_two_rows<__nv_bfloat16, 12>(xrow(r), xrow(r2), nvec, qrow_ptr(r), qrow_ptr(r2), lane, s0,
+                                                        s1);
+            publish(r, s0);
+            publish(r2, s1);
+          } else {
+            publish(r, qrow::quantize_row<__nv_bfloat16, 12>(xrow(r), nvec, qrow_ptr(r), lane));
+          }
+        } else {
+          publish(r, qrow::quantize_row<__nv_bfloat16, 0>(xrow(r), nvec, qrow_ptr(r), lane));
+          if (r2 < p.M) publish(r2, qrow::quantize_row<__nv_bfloat16, 0>(xrow(r2), nvec, qrow_ptr(r2), lane));
+        }
+      }
+    }
     for (int tile = unit; ok && tile < p.num_tiles; tile += num_units, ++local) {
       int mb, nb;
       tile_coords(tile, p, mb, nb);
@@ -349,8 +430,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row0 = mb * kTileM + static_cast<int>(rank) * kBlockM + quarter * 32;
       const int row = row0 + lane;
       float sa = 0.0f;
+      if constexpr (FUSE) {
+        // The scales of this row block were written by other warps of the grid.
+        ok = counter_wait_bounded(&p.sync[mb], static_cast<uint32_t>(min(kBlockM, p.M - mb * kBlockM)), abort_flag,
+                                  p.timeout_ns, p.err, kSiteRowsReady);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+      }
       if constexpr (OUT == GemmOut::kBf16Dequant) {
-        if (row < p.M) sa = __ldg(p.scale_a + row);
+        if (row < p.M) sa = FUSE ? p.scale_out[row] : __ldg(p.scale_a + row);
         // This tile's scale_w and bias, staged once for all epilogue warps
         // (the first barrier: every warp is done with the previous tile's).
         named_barrier_sync(1, 32 * kEpiWarps);
@@ -444,6 +532,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
   }
+  if constexpr (FUSE) {
+    // Every CTA is done with the row-block counters: the last one out
+    // returns them to zero for the next call.
+    if (threadIdx.x == 0) {
+      __threadfence();
+      const uint32_t prev = atomicAdd(&p.sync[p.m_tiles], 1u);
+      if (prev == gridDim.x - 1) {
+        for (int i = 0; i <= p.m_tiles; ++i) p.sync[i] = 0u;
+        __threadfence();
+      }
+    }
+  }
   if constexpr (PAIR) cluster_sync_all();
   if (warp == 1) {
     tc_fence_after_sync();
@@ -513,8 +613,9 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem, const void
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, GemmOut OUT, bool PAIR>
+template <int BN, GemmOut OUT, bool PAIR, bool FUSE>
 cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t stream) {
+  static_assert(!(FUSE && PAIR), "the fused linear layer runs on single CTAs");
   constexpr int kTileM = PAIR ? 2 * kBlockM : kBlockM;
   constexpr int kBRows = PAIR ? BN / 2 : BN;
   CUtensorMap tm_a, tm_b, tm_d;
@@ -545,11 +646,16 @@ cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t 
   p.bias = static_cast<const __nv_bfloat16*>(a.bias);
   p.timeout_ns = a.timeout_ns;
   p.err = nullptr;
+  p.x = static_cast<const __nv_bfloat16*>(a.x);
+  p.ldx = a.ldx;
+  p.xq_out = const_cast<int8_t*>(a.xq);
+  p.scale_out = const_cast<float*>(a.scale_a);
+  p.sync = a.sync;
   cudaError_t e = error_word_address(&p.err);
   if (e != cudaSuccess) return e;
 
   const int smem = smem_bytes(PAIR, BN, cfg.stages);
-  auto kernel = gemm_w8a8_kernel<BN, OUT, PAIR>;
+  auto kernel = gemm_w8a8_kernel<BN, OUT, PAIR, FUSE>;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   // Persistent grid: one CTA (or CTA pair) per tile at most.
@@ -562,13 +668,29 @@ cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t 
   lc.blockDim = dim3(kThreads);
   lc.dynamicSmemBytes = static_cast<size_t>(smem);
   lc.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = PAIR ? 2 : 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  if constexpr (FUSE) {
+    // CTAs wait on rows quantized by other CTAs: all must be resident at
+    // once, which a cooperative launch guarantees (or refuses to launch).
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+  } else {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = PAIR ? 2 : 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+  }
   lc.attrs = attr;
   lc.numAttrs = 1;
+  if (!FUSE && a.overlap_prologue) {
+    // Programmatic dependent launch: the kernel may start while the previous
+    // kernel of the stream (the activation quantizer) finishes; it reads the
+    // weight operand, scale_w and bias early and waits (griddepcontrol.wait)
+    // before the first read of the quantized activations or their scales.
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    lc.numAttrs = 2;
+  }
   e = cudaLaunchKernelEx(&lc, kernel, tm_a, tm_b, tm_d, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -599,23 +721,29 @@ int gemm_max_stages(int block_m, int block_n) {
 cudaError_t launch_gemm(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t stream) {
   const bool bf16 = a.out_kind == GemmOut::kBf16Dequant;
   using O = GemmOut;
+  if (a.fused) {
+    if (!bf16 || cfg.block_m != 128) return cudaErrorInvalidValue;
+    if (cfg.block_n == 256) return launch_typed<256, O::kBf16Dequant, false, true>(a, cfg, stream);
+    if (cfg.block_n == 128) return launch_typed<128, O::kBf16Dequant, false, true>(a, cfg, stream);
+    return cudaErrorInvalidValue;
+  }
   if (cfg.block_m == 256) {
     if (cfg.block_n == 256) {
-      return bf16 ? launch_typed<256, O::kBf16Dequant, true>(a, cfg, stream)
-                  : launch_typed<256, O::kInt32, true>(a, cfg, stream);
+      return bf16 ? launch_typed<256, O::kBf16Dequant, true, false>(a, cfg, stream)
+                  : launch_typed<256, O::kInt32, true, false>(a, cfg, stream);
     }
     if (cfg.block_n == 128) {
-      return bf16 ? launch_typed<128, O::kBf16Dequant, true>(a, cfg, stream)
-                  : launch_typed<128, O::kInt32, true>(a, cfg, stream);
+      return bf16 ? launch_typed<128, O::kBf16Dequant, true, false>(a, cfg, stream)
+                  : launch_typed<128, O::kInt32, true, false>(a, cfg, stream);
     }
   } else if (cfg.block_m == 128) {
     if (cfg.block_n == 256) {
-      return bf16 ? launch_typed<256, O::kBf16Dequant, false>(a, cfg, stream)
-                  : launch_typed<256, O::kInt32, false>(a, cfg, stream);
+      return bf16 ? launch_typed<256, O::kBf16Dequant, false, false>(a, cfg, stream)
+                  : launch_typed<256, O::kInt32, false, false>(a, cfg, stream);
     }
     if (cfg.block_n == 128) {
-      return bf16 ? launch_typed<128, O::kBf16Dequant, false>(a, cfg, stream)
-                  : launch_typed<128, O::kInt32, false>(a, cfg, stream);
+      return bf16 ? launch_typed<128, O::kBf16Dequant, false, false>(a, cfg, stream)
+                  : launch_typed<128, O::kInt32, false, false>(a, cfg, stream);
     }
   }
   return cudaErrorInvalidValue;

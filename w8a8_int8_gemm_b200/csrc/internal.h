@@ -28,7 +28,21 @@ struct GemmArgs {
   int64_t M, N, K;
   GemmOut out_kind;
   uint64_t timeout_ns;
+  // The fused linear layer: quantize x [M, K] (bf16, row stride ldx) into
+  // xq / scale_a inside the GEMM kernel (xq and scale_a are then outputs);
+  // sync is the zeroed row-block counter workspace (linear_sync_words(M)).
+  bool fused = false;
+  // Launch as a programmatic dependent of the previous kernel (only when
+  // that kernel is this library's quantizer writing xq / scale_a and
+  // nothing else: the GEMM reads wq, scale_w and bias before it waits).
+  bool overlap_prologue = false;
+  const void* x = nullptr;
+  int64_t ldx = 0;
+  uint32_t* sync = nullptr;
 };
+
+// 32-bit words of the counter workspace of the fused linear layer.
+inline int64_t linear_sync_words(int64_t M) { return (M + 127) / 128 + 1; }
 
 cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq,
                                 float* scale, cudaStream_t stream);

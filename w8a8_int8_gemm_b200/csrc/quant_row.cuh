@@ -1,0 +1,268 @@
+// quant_row.cuh -- one warp quantizes one row (symmetric absmax, int8).
+//
+// Shared by the standalone row quantizers (quant.cu) and the fused linear
+// kernel (gemm_sm100.cu), which quantizes activation rows inside the GEMM.
+// The rule, and why the product shortcut decides the same codes as the
+// IEEE division, are stated at the top of quant.cu.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+namespace w8a8 {
+namespace qrow {
+
+template <typename T>
+struct Vec;
+
+// 8 bf16 per 16 bytes.
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int kElems = 8;
+  __device__ __forceinline__ static void unpack(const uint4& v, float (&f)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+};
+
+// 4 fp32 per 16 bytes.
+template <>
+struct Vec<float> {
+  static constexpr int kElems = 4;
+  __device__ __forceinline__ static void unpack(const uint4& v, float (&f)[4]) {
+    f[0] = __uint_as_float(v.x);
+    f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z);
+    f[3] = __uint_as_float(v.w);
+  }
+};
+
+// max |x| over one 16-byte vector, as a float.
+template <typename T>
+__device__ __forceinline__ float vec_absmax(const uint4& v);
+
+template <>
+__device__ __forceinline__ float vec_absmax<__nv_bfloat16>(const uint4& v) {
+  // |x| of bf16 pairs by clearing the sign bits, then packed bf16 maxima.
+  const uint32_t w[4] = {v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu, v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu};
+  __nv_bfloat162 m01 = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&w[0]),
+                               *reinterpret_cast<const __nv_bfloat162*>(&w[1]));
+  __nv_bfloat162 m23 = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&w[2]),
+                               *reinterpret_cast<const __nv_bfloat162*>(&w[3]));
+  const __nv_bfloat162 m = __hmax2(m01, m23);
+  const uint32_t mb = *reinterpret_cast<const uint32_t*>(&m);
+  return fmaxf(__uint_as_float(mb << 16), __uint_as_float(mb & 0xFFFF0000u));
+}
+
+template <>
+__device__ __forceinline__ float vec_absmax<float>(const uint4& v) {
+  return fmaxf(fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y))),
+               fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w))));
+}
+
+__device__ __forceinline__ int clamp127(int q) { return max(-127, min(127, q)); }
+
+// Low bytes of four 32-bit words, packed into one word (word 0 lowest).
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+template <int E>
+__device__ __forceinline__ void store_words(const uint32_t (&w)[E], int8_t* dst) {
+  if constexpr (E == 8) {
+    *reinterpret_cast<uint2*>(dst) =
+        make_uint2(pack_low_bytes(w[0], w[1], w[2], w[3]), pack_low_bytes(w[4], w[5], w[6], w[7]));
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pack_low_bytes(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// The exact path: every element as rne(fl32(x / s)) clamped to +-127.
+template <typename T>
+__device__ __noinline__ void quantize_vec_div(uint4 v, float s, int8_t* dst) {
+  constexpr int E = Vec<T>::kElems;
+  float f[E];
+  Vec<T>::unpack(v, f);
+  uint32_t q[E];
+#pragma unroll
+  for (int i = 0; i < E; ++i) q[i] = static_cast<uint32_t>(clamp127(__float2int_rn(__fdiv_rn(f[i], s))));
+  store_words<E>(q, dst);
+}
+
+// The product path with the tie check described at the top of quant.cu:
+// m = fl(x*r + 1.5*2^23) rounds the exact product x*r to an integer (ties to
+// even; 1.5*2^23 is even) in one fused multiply-add, so m - 1.5*2^23 is that
+// integer n and the low byte of m's bit pattern is its int8 code; the
+// residual x*r - n (one more fused multiply-add, rounding error <= 2^-25)
+// flags elements within 2^-15 of a half-integer, whose vector is redone
+// with IEEE division.
+template <typename T>
+__device__ __forceinline__ void quantize_vec(const uint4& v, float s, float r, bool fast, int8_t* dst) {
+  constexpr int E = Vec<T>::kElems;
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  if (fast) {
+    float f[E];
+    Vec<T>::unpack(v, f);
+    uint32_t q[E];
+    bool near_tie = false;
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      const float m = __fmaf_rn(f[i], r, kRound);  // rne(x*r) + 1.5 * 2^23, exactly
+      const float n = __fsub_rn(m, kRound);        // rne(x*r)
+      near_tie |= fabsf(__fmaf_rn(f[i], r, -n)) >= 0.499969482421875f;  // 0.5 - 2^-15
+      q[i] = __float_as_uint(m);                   // low byte = int8 code
+    }
+    if (!near_tie) {
+      store_words<E>(q, dst);
+      return;
+    }
+  }
+  quantize_vec_div<T>(v, s, dst);
+}
+
+struct RowScale {
+  float s, r;
+  bool zero, fast;
+};
+
+__device__ __forceinline__ RowScale row_scale(float amax) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  RowScale rs;
+  rs.s = __fdiv_rn(amax, 127.0f);
+  rs.zero = (rs.s == 0.0f);  // all-zero row (or an fp32 row whose scale underflows): codes 0
+  rs.r = rs.zero ? 0.0f : __frcp_rn(rs.s);
+  rs.fast = !rs.zero && rs.s >= 1.17549435e-38f && isfinite(rs.r);
+  return rs;
+}
+
+template <int E>
+__device__ __forceinline__ void store_zero(int8_t* dst) {
+  if constexpr (E == 8) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = 0u;
+  }
+}
+
+// One warp quantizes row `xr` (nvec 16-byte vectors) into `qr` and returns
+// the row's scale in every lane.  VPL > 0: rows of up to 32 * VPL vectors,
+// all loads issued at once and the row kept in registers; VPL == 0: any
+// length, an absmax pass and a second pass that reads the row again.
+template <typename T, int VPL>
+__device__ __forceinline__ float quantize_row(const uint4* __restrict__ xr, int nvec, int8_t* __restrict__ qr,
+                                              int lane) {
+  constexpr int E = Vec<T>::kElems;
+  if constexpr (VPL > 0) {
+    uint4 c[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int v = lane + 32 * i;
+      c[i] = v < nvec ? __ldg(xr + v) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) amax = fmaxf(amax, vec_absmax<T>(c[i]));
+    const RowScale rs = row_scale(amax);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int v = lane + 32 * i;
+      if (v < nvec) {
+        if (rs.zero) {
+          store_zero<E>(qr + E * v);
+        } else {
+          quantize_vec<T>(c[i], rs.s, rs.r, rs.fast, qr + E * v);
+        }
+      }
+    }
+    return rs.s;
+  } else {
+    // pass 1: absmax, eight 16-byte loads per lane in flight
+    float amax = 0.0f;
+    int v = lane;
+    for (; v + 224 < nvec; v += 256) {
+      uint4 a[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a[i] = __ldg(xr + v + 32 * i);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, vec_absmax<T>(a[i]));
+    }
+    for (; v < nvec; v += 32) amax = fmaxf(amax, vec_absmax<T>(__ldg(xr + v)));
+    const RowScale rs = row_scale(amax);
+    // pass 2: codes
+    v = lane;
+    for (; v + 96 < nvec; v += 128) {
+      uint4 a[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = __ldg(xr + v + 32 * i);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (rs.zero) {
+          store_zero<E>(qr + E * (v + 32 * i));
+        } else {
+          quantize_vec<T>(a[i], rs.s, rs.r, rs.fast, qr + E * (v + 32 * i));
+        }
+      }
+    }
+    for (; v < nvec; v += 32) {
+      if (rs.zero) {
+        store_zero<E>(qr + E * v);
+      } else {
+        quantize_vec<T>(__ldg(xr + v), rs.s, rs.r, rs.fast, qr + E * v);
+      }
+    }
+    return rs.s;
+  }
+}
+
+// Two rows by one warp, both rows' loads in flight together (rows of up to
+// 32 * VPL vectors, kept in registers): twice the memory parallelism of
+// quantize_row for a warp that has several rows to do.  Scales are returned
+// in s0 / s1 (every lane).
+template <typename T, int VPL>
+__device__ __forceinline__ void quantize_two_rows(const uint4* __restrict__ x0, const uint4* __restrict__ x1,
+                                                  int nvec, int8_t* __restrict__ q0, int8_t* __restrict__ q1,
+                                                  int lane, float& s0, float& s1) {
+  constexpr int E = Vec<T>::kElems;
+  uint4 c0[VPL], c1[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int v = lane + 32 * i;
+    c0[i] = v < nvec ? __ldg(x0 + v) : make_uint4(0u, 0u, 0u, 0u);
+    c1[i] = v < nvec ? __ldg(x1 + v) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    a0 = fmaxf(a0, vec_absmax<T>(c0[i]));
+    a1 = fmaxf(a1, vec_absmax<T>(c1[i]));
+  }
+  const RowScale r0 = row_scale(a0);
+  const RowScale r1 = row_scale(a1);
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int v = lane + 32 * i;
+    if (v < nvec) {
+      if (r0.zero) {
+        store_zero<E>(q0 + E * v);
+      } else {
+        quantize_vec<T>(c0[i], r0.s, r0.r, r0.fast, q0 + E * v);
+      }
+      if (r1.zero) {
+        store_zero<E>(q1 + E * v);
+      } else {
+        quantize_vec<T>(c1[i], r1.s, r1.r, r1.fast, q1 + E * v);
+      }
+    }
+  }
+  s0 = r0.s;
+  s1 = r1.s;
+}
+
+}  // namespace qrow
+}  // namespace w8a8

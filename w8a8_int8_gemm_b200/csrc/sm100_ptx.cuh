@@ -20,6 +20,7 @@ enum WaitSite : int {
   kSiteEpiTmemFull = 4,     // epilogue waiting for a finished accumulator
   kSiteDrain = 5,           // teardown waiting for in-flight copies / MMAs
   kSiteSelfTest = 6,        // the timeout self-test
+  kSiteRowsReady = 7,       // fused linear: waiting for a block of quantized rows
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -108,6 +109,59 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
                                           uint64_t timeout_ns, int* err, int site) {
   const bool ok = mbar_wait_bounded(bar, parity, abort, timeout_ns, err, site);
   return __all_sync(0xffffffffu, ok);
+}
+
+// --------------------------------------- programmatic dependent launch
+
+// Lets the next kernel of the stream, if it was launched as a programmatic
+// dependent, start before this grid finishes.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Waits until the grids this one depends on have completed and their
+// memory is visible (returns at once when there are none).
+__device__ __forceinline__ void pdl_wait_prerequisites() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// ------------------------------------------- cross-CTA global counters
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_gpu_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Orders this thread's generic-proxy global writes with later async-proxy
+// (TMA) accesses to global memory, and an acquire of such writes with this
+// thread's later TMA reads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Wait until *p >= need (acquire), for at most timeout_ns; like
+// mbar_wait_bounded it gives up early when *abort is set.
+__device__ __forceinline__ bool counter_wait_bounded(const uint32_t* p, uint32_t need, volatile int* abort,
+                                                     uint64_t timeout_ns, int* err, int site) {
+  if (ld_acquire_gpu(p) >= need) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    __nanosleep(32);
+    if (ld_acquire_gpu(p) >= need) return true;
+    if ((i & 15u) == 0) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > timeout_ns) {
+        record_timeout(err, site);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
 }
 
 // ----------------------------------------------------------------- TMA
