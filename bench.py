@@ -65,6 +65,23 @@ def dist_env() -> tuple[int, int, int]:
             int(os.environ.get("LOCAL_RANK", "0")))
 
 
+def rank_token_rows(M: int, rank: int) -> slice:
+    """Rows of the (seeded) token stream that rank `rank` processes: every
+    rank runs its own batch of M tokens (weak scaling); tokens are
+    independent, so no rank needs another rank's data."""
+    return slice(rank * M, (rank + 1) * M)
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """The largest `value` over all ranks (the timed region's wall time)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def measured_peaks() -> dict:
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -263,7 +280,7 @@ def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
     M, N, K = wl.M, wl.N, wl.K
     if wl.kind != "linear":
         raise SystemExit(f"workload {wl.name} gives int8 codes; bench the linear-layer workloads")
-    d = workloads.make(wl, rows=slice(rank * M, (rank + 1) * M))
+    d = workloads.make(wl, rows=rank_token_rows(M, rank))
     w32 = torch.from_numpy(d["w"]).to(dev)
     x_host = torch.from_numpy(d["x"].view(np.int16)).view(torch.bfloat16)
     bias = torch.from_numpy(d["bias"].view(np.int16)).view(torch.bfloat16).to(dev)
@@ -342,11 +359,7 @@ def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
     clocks = sampler.stop()
     if world > 1:
         torch.distributed.barrier()
-    elapsed_ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), dev)
     code = w8.w8a8_read_device_error()
     if code != 0:
         raise SystemExit(f"a kernel wait timed out in the timed region (site {code})")
