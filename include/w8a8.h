@@ -72,7 +72,8 @@ typedef enum {
     W8A8_ERR_UNSUPPORTED_DEVICE = 3,  /* current device is not sm_100 */
     W8A8_ERR_LAUNCH = 4,              /* CUDA refused the launch */
     W8A8_ERR_TIMEOUT = 5,             /* a kernel's bounded wait ran out (see w8a8_read_device_error) */
-    W8A8_ERR_CUDA = 6                 /* another CUDA runtime error */
+    W8A8_ERR_CUDA = 6,                /* another CUDA runtime error */
+    W8A8_ERR_SCRATCH_LIMIT = 7        /* w8a8_linear_noalloc: the problem needs more than its fixed scratch */
 } w8a8_status;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -154,6 +155,30 @@ W8A8_API w8a8_status w8a8_linear_fused(const void* x, const int8_t* wq, const fl
 
 /* Number of uint32 words of ws_sync for M tokens (M >= 0): ceil(M/128) + 1. */
 W8A8_API int64_t w8a8_linear_sync_words(int64_t M);
+
+/*
+ * w8a8_linear for callers that cannot allocate device memory (the paper
+ * has no counterpart: this is a deployment variant).  Some callers cannot
+ * give the layer a workspace and must not make it allocate one: a runtime
+ * whose device memory is all pre-reserved by another framework's pool, a
+ * latency-critical path where cudaMalloc / cudaFree would synchronize the
+ * device, or a plugin interface that passes only inputs and outputs.
+ *   Arguments as in w8a8_linear, without ws_xq / ws_scale_a: the quantized
+ *   activations and their scales go to one fixed 32 MiB array compiled into
+ *   the library (held by every GPU that loads the library until exit).
+ * Limit: the int8 codes (M*K bytes, rounded up to 256) plus 4*M bytes of
+ * scales must fit in 32 MiB (e.g. 9216 x 3072, 4096 x 8192); larger
+ * problems return W8A8_ERR_SCRATCH_LIMIT and launch nothing.  The call
+ * allocates nothing (no cudaMalloc / cudaFree).  Its first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress, with that
+ * device current); make that first call before any stream capture.  All
+ * calls share the one array, which keeps the last call's contents: calls
+ * that overlap on the GPU (other streams, other host threads) race on it.
+ * Nothing in it needs to start at zero.  Results are bit-identical to
+ * w8a8_linear.
+ */
+W8A8_API w8a8_status w8a8_linear_noalloc(const void* x, const int8_t* wq, const float* scale_w, const void* bias,
+                                         void* out, int64_t M, int64_t N, int64_t K, w8a8_stream_t stream);
 
 /*
  * The GEMM without the epilogue: raw int32 accumulators

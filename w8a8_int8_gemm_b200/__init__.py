@@ -27,6 +27,7 @@ __all__ = [
     "w8a8_status_string", "w8a8_abi_version",
     "w8a8_quantize_act", "w8a8_quantize_weight", "w8a8_gemm", "w8a8_gemm_ex",
     "w8a8_gemm_i32", "w8a8_gemm_i32_ex", "w8a8_linear", "w8a8_linear_fused", "w8a8_linear_sync_words",
+    "w8a8_linear_noalloc",
     "w8a8_select_config",
     "w8a8_read_device_error", "w8a8_set_wait_timeout_ns", "w8a8_selftest_wait_timeout",
 ]
@@ -73,6 +74,7 @@ def _load() -> ctypes.CDLL:
         "w8a8_linear": ([p, p, p, p, p, p, p, i64, i64, i64, p], ctypes.c_int),
         "w8a8_linear_fused": ([p, p, p, p, p, p, p, p, i64, i64, i64, p], ctypes.c_int),
         "w8a8_linear_sync_words": ([i64], i64),
+        "w8a8_linear_noalloc": ([p, p, p, p, p, i64, i64, i64, p], ctypes.c_int),
         "w8a8_select_config": ([i64, i64, i64, ctypes.POINTER(GemmConfig)], ctypes.c_int),
         "w8a8_read_device_error": ([ctypes.POINTER(i32), i32], ctypes.c_int),
         "w8a8_set_wait_timeout_ns": ([i64], ctypes.c_int),
@@ -329,6 +331,31 @@ def w8a8_linear_fused(x, wq, scale_w, bias=None, out=None, ws_xq=None, ws_scale_
     _check(_lib.w8a8_linear_fused(_ptr(x), _ptr(wq), _ptr(scale_w), _ptr(bias), _ptr(out), _ptr(ws_xq),
                                   _ptr(ws_scale_a), _ptr(ws_sync), M, N, K, _stream(stream, dev)),
            "w8a8_linear_fused")
+    return out
+
+
+def w8a8_linear_noalloc(x, wq, scale_w, bias=None, out=None, stream=None):
+    """w8a8_linear without a workspace, for callers that cannot allocate
+    device memory: the quantized activations live in one fixed 32 MiB array
+    inside the library (see include/w8a8.h for the limit and for why
+    overlapping calls race).  `out` must be given by such callers; if it is
+    omitted, this wrapper allocates it with torch for convenience."""
+    _need(x, "x", torch.bfloat16, 2)
+    M, K = x.shape
+    _need(wq, "wq", torch.int8, 2)
+    N = wq.shape[0]
+    if wq.shape[1] != K:
+        raise ValueError(f"inner dimensions differ: x has K={K}, wq has K={wq.shape[1]}")
+    _need_contig(x, "x", torch.bfloat16, (M, K))
+    _need_contig(wq, "wq", torch.int8, (N, K))
+    _need_contig(scale_w, "scale_w", torch.float32, (N,))
+    if bias is not None:
+        _need_contig(bias, "bias", torch.bfloat16, (N,))
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need_contig(out, "out", torch.bfloat16, (M, N))
+    _check(_lib.w8a8_linear_noalloc(_ptr(x), _ptr(wq), _ptr(scale_w), _ptr(bias), _ptr(out), M, N, K,
+                                    _stream(stream, x.device)), "w8a8_linear_noalloc")
     return out
 
 

@@ -179,6 +179,7 @@ const char* w8a8_status_string(int status) {
     case W8A8_ERR_LAUNCH: return "kernel launch failed";
     case W8A8_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
     case W8A8_ERR_CUDA: return "CUDA runtime error";
+    case W8A8_ERR_SCRATCH_LIMIT: return "problem exceeds the fixed scratch of w8a8_linear_noalloc (32 MiB)";
     default: return "unknown status";
   }
 }
