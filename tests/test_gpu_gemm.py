@@ -65,6 +65,22 @@ def test_i32_every_config(w8, cfg):
     assert np.array_equal(_i32(w8, xq, wq, config=cfg), oracle.gemm_i64(xq, wq))
 
 
+# Grids that leave a short last round: its tiles are split into two half-width
+# items (e.g. 12 tiles on 5 CTAs: 10 whole tiles, then 2 tiles as 4 halves).
+TAIL_CASES = [((300, 776, 656), 5), ((300, 776, 656), 9), ((129, 520, 1040), 4), ((260, 1032, 272), 13)]
+
+
+@pytest.mark.parametrize("shape,grid", TAIL_CASES, ids=lambda v: str(v))
+def test_tail_halves_i32_and_bf16(w8, shape, grid):
+    M, N, K = shape
+    cfg = dict(block_m=128, block_n=256, stages=4, grid=grid, raster_group=1)
+    rng = np.random.default_rng(M + grid)
+    xq, wq = _codes(rng, M, K), _codes(rng, N, K)
+    assert np.array_equal(_i32(w8, xq, wq, config=cfg), oracle.gemm_i64(xq, wq))
+    got, want = _bf16_gemm_case(w8, M, N, K, M * 3 + grid, True, cfg)
+    assert bf16_ulp_diff(got, want).max() <= 1
+
+
 def test_i32_identity_and_extremes(w8):
     """Closed forms: identity weight gives 127 * xq; all +-127 rows at K = 12288."""
     rng = np.random.default_rng(1)

@@ -61,6 +61,10 @@ constexpr int kBarrierBytes = 256;
 struct Params {
   int M, N, K;
   int m_tiles, n_tiles, k_blocks, num_tiles;
+  // Work items: tiles [0, full_tiles) whole; when the last round of tiles
+  // would leave CTAs idle, each remaining tile is done as two half-width
+  // items (block_n / 2 columns each), so work_items = full_tiles + 2 * tail.
+  int full_tiles, work_items;
   int raster_group;
   int stages;
   const float* scale_a;
@@ -91,6 +95,21 @@ int smem_bytes(bool pair, int bn, int stages) {
   const int b_rows = pair ? bn / 2 : bn;
   return 1024 + stages * (a_stage_bytes() + b_rows * kBlockK) + kEpiWarps * kEpiBufBytes + params_bytes(bn) +
          kBarrierBytes;
+}
+
+__device__ __forceinline__ void tile_coords(int tile, const Params& p, int& mb, int& nb);
+
+// Work item -> output tile (mb, nb) and half (-1: the whole tile, 0 / 1:
+// the left / right block_n / 2 columns of a tail tile).
+__device__ __forceinline__ void item_coords(int item, const Params& p, int& mb, int& nb, int& hb) {
+  if (item < p.full_tiles) {
+    tile_coords(item, p, mb, nb);
+    hb = -1;
+  } else {
+    const int r = item - p.full_tiles;
+    tile_coords(p.full_tiles + (r >> 1), p, mb, nb);
+    hb = r & 1;
+  }
 }
 
 __device__ __forceinline__ void tile_coords(int tile, const Params& p, int& mb, int& nb) {
@@ -153,7 +172,8 @@ __device__ __forceinline__ void dequant_32(const uint32_t (&v)[32], float sa, co
 template <int BN, GemmOut OUT, bool PAIR, bool FUSE>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                     const __grid_constant__ CUtensorMap tm_d, const Params p) {
+                     const __grid_constant__ CUtensorMap tm_b_half, const __grid_constant__ CUtensorMap tm_d,
+                     const Params p) {
   constexpr int kTileM = PAIR ? 2 * kBlockM : kBlockM;  // rows of the output tile
   constexpr int kBRows = PAIR ? BN / 2 : BN;             // rows of B this CTA loads
   constexpr uint32_t kA = a_stage_bytes();
@@ -161,6 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kTxBytes = (PAIR ? 2 : 1) * (kA + kB);
   constexpr uint32_t kTmemCols = 2 * BN;  // two accumulator buffers; 256 or 512 (power of two)
   constexpr uint32_t kIdesc = make_idesc_i8(kTileM, BN);
+  constexpr uint32_t kIdescHalf = make_idesc_i8(kTileM, BN / 2);  // half-width tail items
   constexpr int kEpiArrivals = (PAIR ? 2 : 1) * kEpiWarps;
 
   extern __shared__ uint8_t smem_raw[];
@@ -201,6 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     prefetch_tensormap(&tm_a);
     prefetch_tensormap(&tm_b);
+    if (p.work_items != p.num_tiles) prefetch_tensormap(&tm_b_half);
     prefetch_tensormap(&tm_d);
   }
   if constexpr (PAIR) {
@@ -233,11 +255,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Both operands are read again by other tiles: keep them in L2 ahead of
     // the streamed output.
     const uint64_t keep = l2_policy_evict_last();
-    for (int tile = unit; ok && tile < p.num_tiles; tile += num_units) {
-      int mb, nb;
-      tile_coords(tile, p, mb, nb);
+    for (int item = unit; ok && item < p.work_items; item += num_units) {
+      int mb, nb, hb;
+      item_coords(item, p, mb, nb, hb);
       const int a_row = mb * kTileM + static_cast<int>(rank) * kBlockM;
-      const int b_row = nb * BN + static_cast<int>(rank) * kBRows;
+      const int b_row = nb * BN + (hb < 0 ? static_cast<int>(rank) * kBRows : hb * (BN / 2));
+      // a half-width item loads half of B's rows, through the tensor map with half-height boxes
+      const CUtensorMap* map_b = hb < 0 ? &tm_b : &tm_b_half;
+      const uint32_t tx_bytes = hb < 0 ? kTxBytes : kA + kB / 2;
       for (int kb = 0; kb < p.k_blocks; ++kb) {
         ok = warp_wait(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns, p.err, kSiteProducerEmpty);
         if (!ok) break;
@@ -249,8 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (fills == 0) pdl_wait_prerequisites();  // A may be written by the kernel before this one
             tma_load_2d_pair_hint(sA + stage * kA, &tm_a, bar, kb * kBlockK, a_row, keep);
           } else {
-            mbar_arrive_expect_tx(&full[stage], kTxBytes);
-            tma_load_2d_hint(sB + stage * kB, &tm_b, &full[stage], kb * kBlockK, b_row, keep);
+            mbar_arrive_expect_tx(&full[stage], tx_bytes);
+            tma_load_2d_hint(sB + stage * kB, map_b, &full[stage], kb * kBlockK, b_row, keep);
             if constexpr (!FUSE) {
               if (fills == 0) pdl_wait_prerequisites();  // A may be written by the kernel before this one
               tma_load_2d_hint(sA + stage * kA, &tm_a, &full[stage], kb * kBlockK, a_row, keep);
@@ -305,7 +330,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
-      for (int tile = unit; ok && tile < p.num_tiles; tile += num_units, ++local) {
+      for (int item = unit; ok && item < p.work_items; item += num_units, ++local) {
+        const uint32_t idesc = item < p.full_tiles ? kIdesc : kIdescHalf;
         const int buf = local & 1;
         const uint32_t tphase = static_cast<uint32_t>(local >> 1) & 1u;
         ok = warp_wait(&tempty[buf], tphase ^ 1u, abort_flag, p.timeout_ns, p.err, kSiteMmaTmemEmpty);
@@ -325,9 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               // per K=32 slice inside the 128-byte swizzled row.
               const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
               if constexpr (PAIR) {
-                mma_i8_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc, acc);
+                mma_i8_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, acc);
               } else {
-                mma_i8(d_tmem, a_desc + 2 * k, b_desc + 2 * k, kIdesc, acc);
+                mma_i8(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, acc);
               }
             }
             if constexpr (PAIR) {
@@ -372,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // quarter a warp may address) and columns half * BN/2 .. +BN/2 of the
     // accumulator, 32 columns at a time, loading the next 32 while it
     // converts the current ones.
-    constexpr int kSub = BN / 2 / 32;                                       // 32-column loads per tile
+    constexpr int kSub = BN / 2 / 32;  // 32-column loads per warp for a whole tile (half-width items: kSub / 2)
     constexpr int kSubPerStore = (OUT == GemmOut::kBf16Dequant) ? 2 : 1;    // loads per 128-byte row block
     const int e = warp - 2;
     const int quarter = warp & 3;
@@ -418,9 +444,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    for (int tile = unit; ok && tile < p.num_tiles; tile += num_units, ++local) {
-      int mb, nb;
-      tile_coords(tile, p, mb, nb);
+    for (int item = unit; ok && item < p.work_items; item += num_units, ++local) {
+      int mb, nb, hb;
+      item_coords(item, p, mb, nb, hb);
+      const int tile_n = hb < 0 ? BN : BN / 2;           // columns of this item
+      const int col_base = nb * BN + (hb < 0 ? 0 : hb * (BN / 2));
+      const int nsub = tile_n / 64;                       // this warp's 32-column loads
       const int buf = local & 1;
       const uint32_t tphase = static_cast<uint32_t>(local >> 1) & 1u;
       ok = warp_wait(&tfull[buf], tphase, abort_flag, p.timeout_ns, p.err, kSiteEpiTmemFull);
@@ -442,25 +471,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         // This tile's scale_w and bias, staged once for all epilogue warps
         // (the first barrier: every warp is done with the previous tile's).
         named_barrier_sync(1, 32 * kEpiWarps);
-        for (int i = e * 32 + lane; i < BN; i += 32 * kEpiWarps) {
-          const int n = nb * BN + i;
+        for (int i = e * 32 + lane; i < tile_n; i += 32 * kEpiWarps) {
+          const int n = col_base + i;
           ps_w[i] = n < p.N ? __ldg(p.scale_w + n) : 0.0f;
           ps_b[i] = (n < p.N && p.bias != nullptr) ? __bfloat16_as_ushort(p.bias[n]) : static_cast<uint16_t>(0);
         }
         named_barrier_sync(1, 32 * kEpiWarps);
       }
       const uint32_t t_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                              static_cast<uint32_t>(buf * BN + half * (BN / 2));
+                              static_cast<uint32_t>(buf * BN + half * (tile_n / 2));
 
       uint32_t va[32], vb[32];
       tmem_load_32cols_async(t_base, va);
       tmem_wait_load(va);
 #pragma unroll
       for (int sc = 0; sc < kSub; ++sc) {
+        if (sc >= nsub) break;  // half-width item
         uint32_t(&cur)[32] = (sc & 1) ? vb : va;
         uint32_t(&nxt)[32] = (sc & 1) ? va : vb;
-        if (sc + 1 < kSub) tmem_load_32cols_async(t_base + 32 * (sc + 1), nxt);
-        if (sc + 1 == kSub) {
+        if (sc + 1 < nsub) tmem_load_32cols_async(t_base + 32 * (sc + 1), nxt);
+        if (sc + 1 == nsub) {
           // The last load of this accumulator buffer has completed.
           tc_fence_before_sync();
           __syncwarp();
@@ -472,8 +502,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        const int cl = half * (BN / 2) + 32 * sc;  // column inside the tile
-        const int col0 = nb * BN + cl - 32 * (sc % kSubPerStore);  // first column of the 128-byte block
+        const int cl = half * (tile_n / 2) + 32 * sc;  // column inside the item
+        const int col0 = col_base + cl - 32 * (sc % kSubPerStore);  // first column of the 128-byte block
         const bool in_range = row0 < p.M && col0 < p.N;
         if (in_range && sc % kSubPerStore == 0) {
           // The previous store from this block must have finished reading it.
@@ -506,12 +536,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tm_d, sbuf, col0, row0);
+            tma_store_2d_hint(&tm_d, sbuf, col0, row0, stream_out);
             bulk_commit_group();
           }
           __syncwarp();
         }
-        if (sc + 1 < kSub) tmem_wait_load(nxt);
+        if (sc + 1 < nsub) tmem_wait_load(nxt);
       }
     }
     if (!ok && PAIR && lane == 0) st_cluster_u32(peer_abort, 1u);
@@ -618,12 +648,14 @@ cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t 
   static_assert(!(FUSE && PAIR), "the fused linear layer runs on single CTAs");
   constexpr int kTileM = PAIR ? 2 * kBlockM : kBlockM;
   constexpr int kBRows = PAIR ? BN / 2 : BN;
-  CUtensorMap tm_a, tm_b, tm_d;
+  CUtensorMap tm_a, tm_b, tm_b_half, tm_d;
   std::memset(&tm_a, 0, sizeof tm_a);
   std::memset(&tm_b, 0, sizeof tm_b);
+  std::memset(&tm_b_half, 0, sizeof tm_b_half);
   std::memset(&tm_d, 0, sizeof tm_d);
   bool ok = encode_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.xq, a.M, a.K, kBlockM, kBlockK) &&
-            encode_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.wq, a.N, a.K, kBRows, kBlockK);
+            encode_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.wq, a.N, a.K, kBRows, kBlockK) &&
+            encode_2d(&tm_b_half, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.wq, a.N, a.K, BN / 2, kBlockK);
   if constexpr (OUT == GemmOut::kBf16Dequant) {
     ok = ok && encode_2d(&tm_d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.out, a.M, a.N, 32, 64);
   } else {
@@ -639,6 +671,8 @@ cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t 
   p.n_tiles = static_cast<int>((a.N + BN - 1) / BN);
   p.k_blocks = static_cast<int>((a.K + kBlockK - 1) / kBlockK);
   p.num_tiles = p.m_tiles * p.n_tiles;
+  p.full_tiles = p.num_tiles;
+  p.work_items = p.num_tiles;
   p.raster_group = cfg.raster_group;
   p.stages = cfg.stages;
   p.scale_a = a.scale_a;
@@ -662,6 +696,13 @@ cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t 
   int units = (PAIR ? cfg.grid / 2 : cfg.grid);
   if (units < 1) units = 1;
   if (units > p.num_tiles) units = p.num_tiles;
+  // Last round: if at most half the CTAs would get a tile, give each of the
+  // remaining tiles to two CTAs as half-width items instead.
+  const int tail = p.num_tiles % units;
+  if (!PAIR && BN == 256 && tail > 0 && 2 * tail <= units) {
+    p.full_tiles = p.num_tiles - tail;
+    p.work_items = p.full_tiles + 2 * tail;
+  }
   cudaLaunchConfig_t lc;
   std::memset(&lc, 0, sizeof lc);
   lc.gridDim = dim3(static_cast<unsigned>(units * (PAIR ? 2 : 1)));
@@ -691,7 +732,7 @@ cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t 
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     lc.numAttrs = 2;
   }
-  e = cudaLaunchKernelEx(&lc, kernel, tm_a, tm_b, tm_d, p);
+  e = cudaLaunchKernelEx(&lc, kernel, tm_a, tm_b, tm_b_half, tm_d, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
