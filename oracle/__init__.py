@@ -72,8 +72,17 @@ class Oracle:
         lib.oracle_epilogue.argtypes = [p, p, p, p, i64, i64, p]
         lib.oracle_epilogue_f64.argtypes = [p, p, p, p, i64, i64, p]
         lib.oracle_linear.argtypes = [p, p, p, p, i64, i64, i64, p, p, p, p, ctypes.c_int]
+        lib.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_to_f64.restype = ctypes.c_double
+        lib.oracle_f32_to_e4m3_rne.argtypes = [ctypes.c_float]
+        lib.oracle_f32_to_e4m3_rne.restype = ctypes.c_uint8
+        lib.oracle_quantize_rows_bf16_fp8.argtypes = [p, i64, i64, i64, p, i64, p]
+        lib.oracle_quantize_rows_f32_fp8.argtypes = [p, i64, i64, i64, p, i64, p]
+        lib.oracle_gemm_fp8_f64.argtypes = [p, p, i64, i64, i64, p]
+        lib.oracle_epilogue_fp8.argtypes = [p, p, p, p, i64, i64, p]
         for fn in ("oracle_quantize_rows_bf16", "oracle_quantize_rows_f32", "oracle_gemm_i64",
-                   "oracle_epilogue", "oracle_epilogue_f64", "oracle_linear"):
+                   "oracle_epilogue", "oracle_epilogue_f64", "oracle_linear", "oracle_quantize_rows_bf16_fp8",
+                   "oracle_quantize_rows_f32_fp8", "oracle_gemm_fp8_f64", "oracle_epilogue_fp8"):
             getattr(lib, fn).restype = ctypes.c_int
         self.lib = lib
         self.path = libpath
@@ -190,6 +199,72 @@ class Oracle:
         return out, xq, sa, acc
 
 
+    # ------------------------------------------------------ fp8 e4m3
+
+    def e4m3_to_f64(self, codes) -> np.ndarray:
+        """E4M3 codes (uint8) -> their values (binary64), element by element in C."""
+        c = _c(codes, np.uint8)
+        out = np.empty(c.shape, np.float64)
+        fi, fo = c.reshape(-1), out.reshape(-1)
+        f = self.lib.oracle_e4m3_to_f64
+        for i in range(fi.size):
+            fo[i] = f(int(fi[i]))
+        return out
+
+    def f32_to_e4m3(self, x) -> np.ndarray:
+        """float32 (|x| <= 448) -> nearest E4M3 code, ties to even (element by element in C)."""
+        a = _c(x, np.float32)
+        out = np.empty(a.shape, np.uint8)
+        fi, fo = a.reshape(-1), out.reshape(-1)
+        f = self.lib.oracle_f32_to_e4m3_rne
+        for i in range(fi.size):
+            fo[i] = f(float(fi[i]))
+        return out
+
+    def quantize_act_fp8(self, x_bits) -> tuple[np.ndarray, np.ndarray]:
+        """Per-token FP8 quantization of bf16 X [M, K]: (codes uint8 [M, K], scale_a [M])."""
+        x = _c(x_bits, np.uint16)
+        M, K = x.shape
+        q = np.empty((M, K), np.uint8)
+        s = np.empty((M,), np.float32)
+        self._check(self.lib.oracle_quantize_rows_bf16_fp8(_ptr(x), M, K, K, _ptr(q), K, _ptr(s)),
+                    "quantize_act_fp8")
+        return q, s
+
+    def quantize_weight_fp8(self, w) -> tuple[np.ndarray, np.ndarray]:
+        """Per-channel FP8 quantization of fp32 W [N, K]: (codes uint8 [N, K], scale_w [N])."""
+        a = _c(w, np.float32)
+        N, K = a.shape
+        q = np.empty((N, K), np.uint8)
+        s = np.empty((N,), np.float32)
+        self._check(self.lib.oracle_quantize_rows_f32_fp8(_ptr(a), N, K, K, _ptr(q), K, _ptr(s)),
+                    "quantize_weight_fp8")
+        return q, s
+
+    def gemm_fp8(self, aq, bq) -> np.ndarray:
+        """acc [M, N] = sum_k e4m3(aq[m,k]) * e4m3(bq[n,k]) in binary64."""
+        a = _c(aq, np.uint8)
+        b = _c(bq, np.uint8)
+        M, K = a.shape
+        N, K2 = b.shape
+        assert K == K2
+        acc = np.empty((M, N), np.float64)
+        self._check(self.lib.oracle_gemm_fp8_f64(_ptr(a), _ptr(b), M, N, K, _ptr(acc)), "gemm_fp8")
+        return acc
+
+    def epilogue_fp8(self, acc, scale_a, scale_w, bias_bits=None) -> np.ndarray:
+        """bf16 bits [M, N] = bf16_rne((fl32(acc) * s_a[m]) * s_w[n] + bias[n])."""
+        c = _c(acc, np.float64)
+        M, N = c.shape
+        sa = _c(scale_a, np.float32)
+        sw = _c(scale_w, np.float32)
+        bias = None if bias_bits is None else _c(bias_bits, np.uint16)
+        out = np.empty((M, N), np.uint16)
+        self._check(self.lib.oracle_epilogue_fp8(_ptr(c), _ptr(sa), _ptr(sw), _ptr(bias), M, N, _ptr(out)),
+                    "epilogue_fp8")
+        return out
+
+
 _default: Oracle | None = None
 
 
@@ -231,3 +306,27 @@ def epilogue_f64(acc, scale_a, scale_w, bias_bits=None):
 
 def linear(x_bits, wq, scale_w, bias_bits=None, nthreads: int | None = None):
     return get().linear(x_bits, wq, scale_w, bias_bits, nthreads)
+
+
+def e4m3_to_f64(codes):
+    return get().e4m3_to_f64(codes)
+
+
+def f32_to_e4m3(x):
+    return get().f32_to_e4m3(x)
+
+
+def quantize_act_fp8(x_bits):
+    return get().quantize_act_fp8(x_bits)
+
+
+def quantize_weight_fp8(w):
+    return get().quantize_weight_fp8(w)
+
+
+def gemm_fp8(aq, bq):
+    return get().gemm_fp8(aq, bq)
+
+
+def epilogue_fp8(acc, scale_a, scale_w, bias_bits=None):
+    return get().epilogue_fp8(acc, scale_a, scale_w, bias_bits)

@@ -28,6 +28,16 @@
  * division).  Rounding-mode dependent calls (nearbyintf) rely on the
  * default round-to-nearest-even mode.
  *
+ * FP8 variant (the paper's comparison baseline and its "native FP8 path" on
+ * B200): the same per-token / per-channel symmetric scheme with OCP FP8
+ * E4M3 codes (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; largest
+ * finite value 448; no infinities):
+ *
+ *   scale[r]  = fl32( max_k |x[r,k]| / 448 )
+ *   q[r,k]    = e4m3_rne( clamp( fl32(x[r,k] / scale[r]), -448, 448 ) )
+ *   acc[m,n]  = sum_k e4m3(q_x[m,k]) * e4m3(q_w[n,k])   (exact, here in binary64)
+ *   out[m,n]  = bf16_rne( fl32( fl32( fl32(acc)*s_a[m] ) * s_w[n] ) + bias[n] )
+ *
  * Parity pins (what this file is checked against, other than itself):
  * brute force and closed forms in the CPU test suite -- numpy float32
  * division and rint for the quantizer, numpy int64 matmul and exact
@@ -64,6 +74,110 @@ uint16_t oracle_f32_to_bf16_rne(float f) {
     /* A carry out of the mantissa moves into the exponent, which is the
      * correct next representable value (up to and including infinity). */
     return (uint16_t)(kept + (uint32_t)round_up);
+}
+
+/* ------------------------------------------------------------ fp8 e4m3 */
+
+/* Value of an E4M3 code: sign, exponent e (bias 7), mantissa m (3 bits);
+ * e == 0 is subnormal (m/8 * 2^-6); 0x7F / 0xFF are NaN. */
+double oracle_e4m3_to_f64(uint8_t c) {
+    int sign = (c >> 7) & 1;
+    int e = (c >> 3) & 0xF;
+    int m = c & 7;
+    double v;
+    if (e == 0xF && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m / 8.0, -6);
+    else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* The E4M3 code nearest to f (ties to the even mantissa), |f| <= 448
+ * (callers clamp).  Found by scanning the 127 non-negative finite codes in
+ * increasing order of value, which is the definition of round to nearest. */
+uint8_t oracle_f32_to_e4m3_rne(float f) {
+    double a = fabs((double)f);
+    uint8_t sign = (f < 0.0f || (f == 0.0f && signbit(f))) ? 0x80 : 0x00;
+    uint8_t best = 0;
+    for (uint8_t c = 1; c < 0x7F; ++c) {        /* codes 0x00..0x7E are finite, increasing */
+        double lo = oracle_e4m3_to_f64((uint8_t)(c - 1));
+        double hi = oracle_e4m3_to_f64(c);
+        if (a < lo) break;
+        if (a >= hi) { best = c; continue; }
+        /* lo <= a < hi */
+        double mid = 0.5 * (lo + hi);
+        if (a > mid) best = c;
+        else if (a < mid) best = (uint8_t)(c - 1);
+        else best = ((c & 1) == 0) ? c : (uint8_t)(c - 1);  /* tie: even code */
+        break;
+    }
+    return (uint8_t)(sign | best);
+}
+
+static void quantize_row_fp8(const float* v, int64_t K, uint8_t* q, float* scale) {
+    float peak = 0.0f;
+    for (int64_t k = 0; k < K; ++k) peak = fmaxf(peak, fabsf(v[k]));
+    float sc = peak / 448.0f;
+    *scale = sc;
+    for (int64_t k = 0; k < K; ++k) {
+        if (sc == 0.0f) { q[k] = 0; continue; }
+        float u = v[k] / sc;         /* one IEEE binary32 division */
+        u = fminf(fmaxf(u, -448.0f), 448.0f);
+        q[k] = oracle_f32_to_e4m3_rne(u);
+    }
+}
+
+/* Per-token FP8 quantizer: bf16 X [M, K] -> E4M3 codes [M, K] + fp32 scales. */
+int oracle_quantize_rows_bf16_fp8(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                                  uint8_t* q, int64_t ldq, float* scale) {
+    if (M < 0 || K < 1 || ldx < K || ldq < K) return 1;
+    float* row = (float*)malloc((size_t)K * sizeof(float));
+    if (!row) return 2;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t k = 0; k < K; ++k) row[k] = oracle_bf16_to_f32(x[m * ldx + k]);
+        quantize_row_fp8(row, K, q + m * ldq, scale + m);
+    }
+    free(row);
+    return 0;
+}
+
+/* Per-channel FP8 quantizer of fp32 W [N, K]. */
+int oracle_quantize_rows_f32_fp8(const float* w, int64_t N, int64_t K, int64_t ldw,
+                                 uint8_t* q, int64_t ldq, float* scale) {
+    if (N < 0 || K < 1 || ldw < K || ldq < K) return 1;
+    for (int64_t n = 0; n < N; ++n) quantize_row_fp8(w + n * ldw, K, q + n * ldq, scale + n);
+    return 0;
+}
+
+/* acc[m, n] = sum_k e4m3(a[m,k]) * e4m3(b[n,k]), in binary64: each product of
+ * two 4-significant-bit values is exact, and for the value ranges of scaled
+ * codes (|q| <= 448, K <= 2^17) the running sum stays exact to far below
+ * binary32's precision. */
+int oracle_gemm_fp8_f64(const uint8_t* a, const uint8_t* b, int64_t M, int64_t N, int64_t K, double* acc) {
+    if (M < 0 || N < 0 || K < 1) return 1;
+    double lut[256];
+    for (int c = 0; c < 256; ++c) lut[c] = oracle_e4m3_to_f64((uint8_t)c);
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double s = 0.0;
+            for (int64_t k = 0; k < K; ++k) s += lut[a[m * K + k]] * lut[b[n * K + k]];
+            acc[m * N + n] = s;
+        }
+    return 0;
+}
+
+/* The epilogue of the FP8 variant: the accumulator rounded once to binary32,
+ * then the same operations as the int8 epilogue. */
+int oracle_epilogue_fp8(const double* acc, const float* scale_a, const float* scale_w,
+                        const uint16_t* bias, int64_t M, int64_t N, uint16_t* out) {
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            float d = (float)acc[m * N + n];      /* the one rounding of the sum */
+            d *= scale_a[m];
+            d *= scale_w[n];
+            float bn = bias ? oracle_bf16_to_f32(bias[n]) : 0.0f;
+            out[m * N + n] = oracle_f32_to_bf16_rne(d + bn);
+        }
+    return 0;
 }
 
 /* --------------------------------------------------- symmetric quantizer */

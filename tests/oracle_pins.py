@@ -349,3 +349,130 @@ ALL_CHECKS = [
     check_epilogue_exact_bound, check_epilogue_bias_optional,
     check_hand_linear, check_linear_identity_weight, check_linear_composition,
 ]
+
+
+# ------------------------------------------------------------ fp8 e4m3
+
+
+def _torch_e4m3(x: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def check_e4m3_decode(orc) -> None:
+    """E4M3 code -> value equals torch's float8_e4m3fn on all 256 codes."""
+    codes = np.arange(256, dtype=np.uint8)
+    mine = orc.e4m3_to_f64(codes)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(mine), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(mine[ok], ref[ok])
+
+
+def check_e4m3_encode(orc) -> None:
+    """value -> E4M3 (RNE) equals torch's conversion, at every midpoint too."""
+    vals = orc.e4m3_to_f64(np.arange(0x7F, dtype=np.uint8))          # non-negative finite codes
+    mids = 0.5 * (vals[:-1] + vals[1:])
+    rng = np.random.default_rng(21)
+    x = np.concatenate([vals, mids, np.nextafter(mids, 0), np.nextafter(mids, 1000),
+                        rng.uniform(0, 448, 3000), rng.uniform(0, 2.0 ** -5, 500)]).astype(np.float32)
+    x = np.concatenate([x, -x])
+    x = x[np.abs(x) <= 448]
+    assert np.array_equal(orc.f32_to_e4m3(x), _torch_e4m3(x))
+
+
+def check_fp8_quant_golden(orc) -> None:
+    """Hand-worked rows (tests/golden/quant_fp8_rows.txt)."""
+    for xs, qs, ss in read_rows("quant_fp8_rows.txt"):
+        x = np.array([float(v) for v in xs], np.float32)
+        q, s = orc.quantize_act_fp8(bf16_bits(x)[None, :])
+        want = np.array([int(v, 16) for v in qs], np.uint8)
+        assert (q[0] == want).all(), f"codes {q[0]} != {want} for {x}"
+        assert s[0] == np.float32(float(ss[0]))
+
+
+def numpy_quantize_fp8(x: np.ndarray):
+    """The FP8 quantizer through numpy float32 division and torch's E4M3 conversion."""
+    x = x.astype(np.float32)
+    amax = np.max(np.abs(x), axis=1)
+    s = (amax / np.float32(448.0)).astype(np.float32)
+    q = np.zeros(x.shape, np.uint8)
+    nz = s > 0
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = (x[nz] / s[nz, None]).astype(np.float32)
+    q[nz] = _torch_e4m3(np.clip(t, -448, 448))
+    return q, s
+
+
+def check_fp8_quant_vs_library(orc) -> None:
+    rng = np.random.default_rng(22)
+    K = 160
+    x = np.concatenate([edge_rows(K, rng), bits_to_float(to_bits(rng.standard_normal((30, K)).astype(np.float32)))])
+    q, s = orc.quantize_act_fp8(to_bits(x))
+    q2, s2 = numpy_quantize_fp8(x)
+    # -0 codes: the library keeps the sign of a negative quotient that rounds to zero
+    assert (s.view(np.uint32) == s2.view(np.uint32)).all()
+    assert (q == q2).all(), np.argwhere(q != q2)[:5]
+    w = (rng.standard_normal((20, 64)) * 0.02).astype(np.float32)
+    wq, sw = orc.quantize_weight_fp8(w)
+    wq2, sw2 = numpy_quantize_fp8(w)
+    assert (sw.view(np.uint32) == sw2.view(np.uint32)).all() and (wq == wq2).all()
+
+
+def check_fp8_quant_invariants(orc) -> None:
+    rng = np.random.default_rng(23)
+    x = bits_to_float(to_bits(rng.standard_normal((32, 200)).astype(np.float32) * 5))
+    q, s = orc.quantize_act_fp8(to_bits(x))
+    arg = np.abs(x).argmax(axis=1)
+    top = q[np.arange(32), arg]
+    assert ((top == 0x7E) | (top == 0xFE)).all(), "the row absmax must map to +-448"
+    vals = orc.e4m3_to_f64(q)
+    # E4M3 keeps 4 significant bits: relative rounding <= 2^-4 (normals) of |x/s|
+    rel = np.abs(vals * s[:, None] - x) / np.maximum(np.abs(x), 1e-30)
+    big = np.abs(x / s[:, None]) >= 2.0 ** -6
+    assert (rel[big] <= 2.0 ** -4 * (1 + 1e-6)).all()
+    q2, s2 = orc.quantize_act_fp8(to_bits(x * np.float32(8.0)))
+    assert (q2 == q).all() and (s2 == s * np.float32(8.0)).all()
+    q3, _ = orc.quantize_act_fp8(to_bits(-x))
+    assert ((q3 ^ q) == 0x80)[x != 0].all()
+
+
+def check_fp8_gemm(orc) -> None:
+    """The FP8 accumulator equals numpy's float64 matmul of the decoded codes;
+    diagonal 1.0 weights select the activations."""
+    rng = np.random.default_rng(24)
+    finite = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    a = rng.choice(finite, (9, 48))
+    b = rng.choice(finite, (7, 48))
+    acc = orc.gemm_fp8(a, b)
+    ref = orc.e4m3_to_f64(a) @ orc.e4m3_to_f64(b).T
+    assert np.allclose(acc, ref, rtol=1e-12, atol=1e-12)
+    ref2 = torch.from_numpy(a).view(torch.float8_e4m3fn).double().numpy() @ \
+        torch.from_numpy(b).view(torch.float8_e4m3fn).double().numpy().T
+    assert np.allclose(acc, ref2, rtol=1e-12, atol=1e-12)
+    eye = np.zeros((48, 48), np.uint8)
+    eye[np.arange(48), np.arange(48)] = 0x38
+    assert np.array_equal(orc.gemm_fp8(a, eye), orc.e4m3_to_f64(a))
+
+
+def check_fp8_epilogue(orc) -> None:
+    """bf16 output within the binary32 + bf16 rounding bound of the exact value."""
+    rng = np.random.default_rng(25)
+    M, N = 12, 16
+    acc = rng.standard_normal((M, N)) * 1e5
+    acc[0, :] = 0.0
+    sa = np.exp(rng.uniform(np.log(1e-4), np.log(1e-1), M)).astype(np.float32)
+    sw = np.exp(rng.uniform(np.log(1e-4), np.log(1e-1), N)).astype(np.float32)
+    bias = to_bits(rng.standard_normal(N).astype(np.float32) * np.float32(0.1))
+    bf = bits_to_float(bias)
+    out = bits_to_float(orc.epilogue_fp8(acc, sa, sw, bias))
+    for m in range(M):
+        for n in range(N):
+            exact = Fraction(float(acc[m, n])) * Fraction(float(sa[m])) * Fraction(float(sw[n])) + Fraction(float(bf[n]))
+            ye = float(exact)
+            prod = abs(float(acc[m, n]) * float(sa[m]) * float(sw[n]))
+            assert abs(float(out[m, n]) - ye) <= U16 * abs(ye) + 5 * U32 * (prod + abs(float(bf[n]))) + 1e-38
+    assert (out[0] == bf).all()
+
+
+ALL_CHECKS += [check_e4m3_decode, check_e4m3_encode, check_fp8_quant_golden, check_fp8_quant_vs_library,
+               check_fp8_quant_invariants, check_fp8_gemm, check_fp8_epilogue]

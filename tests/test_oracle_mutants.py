@@ -31,6 +31,26 @@ MUTANTS = [
     ("bf16 widening shift", "uint32_t u = ((uint32_t)h) << 16;", "uint32_t u = ((uint32_t)h) << 15;"),
     ("zero test on absmax instead of scale", "if (s == 0.0f) { q[k] = 0; continue; }",
      "if (amax == 0.0f) { q[k] = 0; continue; }"),
+    # fp8 e4m3 variant
+    ("e4m3 divisor 447", "float sc = peak / 448.0f;", "float sc = peak / 447.0f;"),
+    ("e4m3 exponent bias 8", "else v = ldexp(1.0 + (double)m / 8.0, e - 7);",
+     "else v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    ("e4m3 subnormal exponent -7", "if (e == 0) v = ldexp((double)m / 8.0, -6);",
+     "if (e == 0) v = ldexp((double)m / 8.0, -7);"),
+    ("e4m3 four mantissa bits", "else v = ldexp(1.0 + (double)m / 8.0, e - 7);",
+     "else v = ldexp(1.0 + (double)m / 16.0, e - 7);"),
+    ("e4m3 sign dropped", "return sign ? -v : v;", "return v;"),
+    ("e4m3 ties to odd", "else best = ((c & 1) == 0) ? c : (uint8_t)(c - 1);",
+     "else best = ((c & 1) == 1) ? c : (uint8_t)(c - 1);"),
+    ("e4m3 ties up", "else best = ((c & 1) == 0) ? c : (uint8_t)(c - 1);", "else best = c;"),
+    ("e4m3 rounds down", "if (a > mid) best = c;", "if (a > hi) best = c;"),
+    ("e4m3 signed peak", "peak = fmaxf(peak, fabsf(v[k]));", "peak = fmaxf(peak, v[k]);"),
+    ("e4m3 gemm transposed weight", "s += lut[a[m * K + k]] * lut[b[n * K + k]];",
+     "s += lut[a[m * K + k]] * lut[b[k * N + n]];"),
+    ("e4m3 gemm wrong reduction index", "s += lut[a[m * K + k]] * lut[b[n * K + k]];",
+     "s += lut[a[m * K + k]] * lut[b[n * K + (K - 1 - k)]];"),
+    ("e4m3 epilogue scale_w twice", "d *= scale_a[m];", "d *= scale_w[n];"),
+    ("e4m3 epilogue dropped bias", "oracle_f32_to_bf16_rne(d + bn);", "oracle_f32_to_bf16_rne(d);"),
 ]
 
 
