@@ -222,6 +222,62 @@ W8A8_API w8a8_status w8a8_gemm_i32_ex(const int8_t* xq, const int8_t* wq, int32_
                              w8a8_stream_t stream);
 
 /*
+ * FP8 variant: OCP E4M3 codes in place of int8.  The paper measures its
+ * int8 kernel against FP8 (abstract: the native FP8 path of datacenter
+ * Blackwell is the comparison baseline); this is that path, with the same
+ * per-token x per-channel scheme and 448 (the largest finite E4M3 value) in
+ * place of 127:
+ *
+ *   scale_a[m] = fl32(max_k |x[m,k]| / 448)
+ *   xq[m,k]    = e4m3_rne(clamp(fl32(x[m,k] / scale_a[m]), -448, 448))
+ *                (0 for a row whose scale is 0; -0 keeps its sign, code 0x80)
+ *   acc[m,n]   = sum_k e4m3(xq[m,k]) * e4m3(wq[n,k])    fp32, tensor cores
+ *   out[m,n]   = bf16_rne((acc[m,n] * scale_a[m]) * scale_w[n] + bias[n])
+ *
+ * (the pages give no FP8 recipe: this reading is the library's definition).
+ * Codes are bytes (uint8_t) in the E4M3 encoding: 1 sign bit, 4 exponent
+ * bits with bias 7, 3 mantissa bits, no infinities, 0x7F / 0xFF NaN (never
+ * produced).  Quantized codes and scales are bit-exact to the definition.
+ * The accumulator: each product of two E4M3 values is exact; the tensor
+ * cores add them in fp32 in an order of their own, so acc differs from the
+ * exact sum by rounding only (the library's tests bound the difference by
+ * K * 2^-23 * sum_k |products|; exact when every partial sum is an fp32
+ * value).  Shapes, strides, alignment and errors as for the int8 calls
+ * (including 16 <= K <= 133144, K % 16 == 0, N % 8 == 0).
+ */
+W8A8_API w8a8_status w8a8_quantize_act_fp8(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                           uint8_t* xq, int64_t ldxq, float* scale_a, w8a8_stream_t stream);
+W8A8_API w8a8_status w8a8_quantize_weight_fp8(const float* w, int64_t N, int64_t K, int64_t ldw,
+                                              uint8_t* wq, int64_t ldwq, float* scale_w, w8a8_stream_t stream);
+
+/* The FP8 GEMM with the dequantization + bias epilogue (tcgen05.mma
+ * kind::f8f6f4): arguments as in w8a8_gemm, with E4M3 codes. */
+W8A8_API w8a8_status w8a8_gemm_fp8(const uint8_t* xq, const uint8_t* wq, const float* scale_a,
+                                   const float* scale_w, const void* bias, void* out,
+                                   int64_t M, int64_t N, int64_t K, w8a8_stream_t stream);
+
+/* The FP8 GEMM without the epilogue: fp32 accumulators acc [M, N] (row
+ * stride N), for checking the accumulation against an exact sum. */
+W8A8_API w8a8_status w8a8_gemm_fp8_f32(const uint8_t* xq, const uint8_t* wq, float* acc,
+                                       int64_t M, int64_t N, int64_t K, w8a8_stream_t stream);
+
+/* The two FP8 GEMMs with an explicit configuration (as w8a8_gemm_ex). */
+W8A8_API w8a8_status w8a8_gemm_fp8_ex(const uint8_t* xq, const uint8_t* wq, const float* scale_a,
+                                      const float* scale_w, const void* bias, void* out,
+                                      int64_t M, int64_t N, int64_t K, const w8a8_gemm_config* cfg,
+                                      w8a8_stream_t stream);
+W8A8_API w8a8_status w8a8_gemm_fp8_f32_ex(const uint8_t* xq, const uint8_t* wq, float* acc,
+                                          int64_t M, int64_t N, int64_t K, const w8a8_gemm_config* cfg,
+                                          w8a8_stream_t stream);
+
+/* The whole FP8 linear layer: w8a8_quantize_act_fp8 into the caller's
+ * workspace (ws_xq uint8 [M, K], ws_scale_a fp32 [M]), then w8a8_gemm_fp8.
+ * Arguments as in w8a8_linear. */
+W8A8_API w8a8_status w8a8_linear_fp8(const void* x, const uint8_t* wq, const float* scale_w, const void* bias,
+                                     void* out, uint8_t* ws_xq, float* ws_scale_a,
+                                     int64_t M, int64_t N, int64_t K, w8a8_stream_t stream);
+
+/*
  * Every wait inside the library's kernels is bounded in time.  When one
  * runs out the kernel records a nonzero code in a device-side error word,
  * finishes its own in-flight copies, frees its tensor memory and exits, so

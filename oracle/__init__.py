@@ -20,6 +20,7 @@ function is "parity unpinned".
 """
 from __future__ import annotations
 
+import concurrent.futures
 import ctypes
 import os
 import subprocess
@@ -241,15 +242,31 @@ class Oracle:
                     "quantize_weight_fp8")
         return q, s
 
-    def gemm_fp8(self, aq, bq) -> np.ndarray:
-        """acc [M, N] = sum_k e4m3(aq[m,k]) * e4m3(bq[n,k]) in binary64."""
+    def gemm_fp8(self, aq, bq, nthreads: int | None = None) -> np.ndarray:
+        """acc [M, N] = sum_k e4m3(aq[m,k]) * e4m3(bq[n,k]) in binary64.
+
+        Row blocks run on host threads (each element is the same
+        single-threaded sum whatever the split)."""
         a = _c(aq, np.uint8)
         b = _c(bq, np.uint8)
         M, K = a.shape
         N, K2 = b.shape
         assert K == K2
         acc = np.empty((M, N), np.float64)
-        self._check(self.lib.oracle_gemm_fp8_f64(_ptr(a), _ptr(b), M, N, K, _ptr(acc)), "gemm_fp8")
+        nt = max(1, min(nthreads or default_threads(), M))
+        bounds = [M * t // nt for t in range(nt + 1)]
+
+        def run(t):
+            r0, r1 = bounds[t], bounds[t + 1]
+            if r1 > r0:
+                self._check(self.lib.oracle_gemm_fp8_f64(_ptr(a[r0:r1]), _ptr(b), r1 - r0, N, K,
+                                                         _ptr(acc[r0:r1])), "gemm_fp8")
+
+        if nt == 1:
+            run(0)
+        else:
+            with concurrent.futures.ThreadPoolExecutor(nt) as ex:
+                list(ex.map(run, range(nt)))
         return acc
 
     def epilogue_fp8(self, acc, scale_a, scale_w, bias_bits=None) -> np.ndarray:

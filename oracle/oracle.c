@@ -91,16 +91,24 @@ double oracle_e4m3_to_f64(uint8_t c) {
     return sign ? -v : v;
 }
 
+/* Values of the non-negative finite codes 0x00..0x7E (filled once). */
+static double e4m3_pos[0x7F];
+static pthread_once_t e4m3_once = PTHREAD_ONCE_INIT;
+static void e4m3_fill(void) {
+    for (int c = 0; c < 0x7F; ++c) e4m3_pos[c] = oracle_e4m3_to_f64((uint8_t)c);
+}
+
 /* The E4M3 code nearest to f (ties to the even mantissa), |f| <= 448
  * (callers clamp).  Found by scanning the 127 non-negative finite codes in
  * increasing order of value, which is the definition of round to nearest. */
 uint8_t oracle_f32_to_e4m3_rne(float f) {
+    pthread_once(&e4m3_once, e4m3_fill);
     double a = fabs((double)f);
     uint8_t sign = (f < 0.0f || (f == 0.0f && signbit(f))) ? 0x80 : 0x00;
     uint8_t best = 0;
     for (uint8_t c = 1; c < 0x7F; ++c) {        /* codes 0x00..0x7E are finite, increasing */
-        double lo = oracle_e4m3_to_f64((uint8_t)(c - 1));
-        double hi = oracle_e4m3_to_f64(c);
+        double lo = e4m3_pos[c - 1];
+        double hi = e4m3_pos[c];
         if (a < lo) break;
         if (a >= hi) { best = c; continue; }
         /* lo <= a < hi */

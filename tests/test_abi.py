@@ -78,6 +78,20 @@ def test_host_validation_without_device(w8):
     assert lib.w8a8_linear_sync_words(128) == 2
     assert lib.w8a8_linear_sync_words(129) == 3
     assert lib.w8a8_linear_sync_words(4096) == 33
+    # the FP8 (E4M3) variant: the same checks
+    assert lib.w8a8_quantize_act_fp8(A, 4, 32, 16, A, 32, A, None) == 1      # ldx < K
+    assert lib.w8a8_quantize_act_fp8(A, 4, 32, 32, A, 40, A, None) == 2      # ldxq not 16-byte
+    assert lib.w8a8_quantize_weight_fp8(A, 4, 24, 24, A, 32, A, None) == 1   # K % 16
+    assert lib.w8a8_quantize_weight_fp8(A, 0, 32, 32, A, 32, A, None) == 0   # empty
+    assert lib.w8a8_gemm_fp8(A, A, A, A, A + 2, A, 4, 8, 32, None) == 2      # misaligned bias
+    assert lib.w8a8_gemm_fp8(A, A, None, A, None, A, 4, 8, 32, None) == 1    # missing scale_a
+    assert lib.w8a8_gemm_fp8_f32(A, A, A, 4, 12, 32, None) == 1             # N % 8
+    assert lib.w8a8_gemm_fp8_f32(A, A, A, 0, 8, 32, None) == 0              # empty
+    assert lib.w8a8_linear_fp8(A, A, A, None, A, A, A, 4, 8, 133152, None) == 1   # K too large
+    assert lib.w8a8_linear_fp8(A, A, A, None, A, A + 4, A, 4, 8, 32, None) == 2   # misaligned ws_xq
+    assert lib.w8a8_linear_fp8(A, A, A, None, A, A, None, 4, 8, 32, None) == 1    # no ws_scale_a
+    cfg = w8.GemmConfig(block_m=256, block_n=256, stages=7, grid=2, raster_group=1)
+    assert lib.w8a8_gemm_fp8_f32_ex(A, A, A, 4, 8, 32, ctypes.byref(cfg), None) == 1  # too many stages
     # explicit configurations
     cfg = w8.GemmConfig(block_m=128, block_n=200, stages=4, grid=1, raster_group=1)
     assert lib.w8a8_gemm_i32_ex(A, A, A, 4, 8, 32, ctypes.byref(cfg), None) == 1

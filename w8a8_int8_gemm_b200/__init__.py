@@ -28,6 +28,8 @@ __all__ = [
     "w8a8_quantize_act", "w8a8_quantize_weight", "w8a8_gemm", "w8a8_gemm_ex",
     "w8a8_gemm_i32", "w8a8_gemm_i32_ex", "w8a8_linear", "w8a8_linear_fused", "w8a8_linear_sync_words",
     "w8a8_linear_noalloc",
+    "w8a8_quantize_act_fp8", "w8a8_quantize_weight_fp8", "w8a8_gemm_fp8", "w8a8_gemm_fp8_ex",
+    "w8a8_gemm_fp8_f32", "w8a8_gemm_fp8_f32_ex", "w8a8_linear_fp8",
     "w8a8_select_config",
     "w8a8_read_device_error", "w8a8_set_wait_timeout_ns", "w8a8_selftest_wait_timeout",
 ]
@@ -75,6 +77,13 @@ def _load() -> ctypes.CDLL:
         "w8a8_linear_fused": ([p, p, p, p, p, p, p, p, i64, i64, i64, p], ctypes.c_int),
         "w8a8_linear_sync_words": ([i64], i64),
         "w8a8_linear_noalloc": ([p, p, p, p, p, i64, i64, i64, p], ctypes.c_int),
+        "w8a8_quantize_act_fp8": ([p, i64, i64, i64, p, i64, p, p], ctypes.c_int),
+        "w8a8_quantize_weight_fp8": ([p, i64, i64, i64, p, i64, p, p], ctypes.c_int),
+        "w8a8_gemm_fp8": ([p, p, p, p, p, p, i64, i64, i64, p], ctypes.c_int),
+        "w8a8_gemm_fp8_ex": ([p, p, p, p, p, p, i64, i64, i64, ctypes.POINTER(GemmConfig), p], ctypes.c_int),
+        "w8a8_gemm_fp8_f32": ([p, p, p, i64, i64, i64, p], ctypes.c_int),
+        "w8a8_gemm_fp8_f32_ex": ([p, p, p, i64, i64, i64, ctypes.POINTER(GemmConfig), p], ctypes.c_int),
+        "w8a8_linear_fp8": ([p, p, p, p, p, p, p, i64, i64, i64, p], ctypes.c_int),
         "w8a8_select_config": ([i64, i64, i64, ctypes.POINTER(GemmConfig)], ctypes.c_int),
         "w8a8_read_device_error": ([ctypes.POINTER(i32), i32], ctypes.c_int),
         "w8a8_set_wait_timeout_ns": ([i64], ctypes.c_int),
@@ -356,6 +365,118 @@ def w8a8_linear_noalloc(x, wq, scale_w, bias=None, out=None, stream=None):
     _need_contig(out, "out", torch.bfloat16, (M, N))
     _check(_lib.w8a8_linear_noalloc(_ptr(x), _ptr(wq), _ptr(scale_w), _ptr(bias), _ptr(out), M, N, K,
                                     _stream(stream, x.device)), "w8a8_linear_noalloc")
+    return out
+
+
+# ------------------------------------------------- FP8 (E4M3) variant
+# E4M3 codes travel as torch.uint8 tensors (view them as
+# torch.float8_e4m3fn to read their values).
+
+
+def _quantize_fp8(fn, what, src, dtype, q, scale, stream):
+    _need(src, "x" if dtype == torch.bfloat16 else "w", dtype, 2)
+    R, K = src.shape
+    if q is None:
+        q = torch.empty((R, K), dtype=torch.uint8, device=src.device)
+    if scale is None:
+        scale = torch.empty((R,), dtype=torch.float32, device=src.device)
+    _need(q, "codes", torch.uint8, 2)
+    if tuple(q.shape) != (R, K):
+        raise ValueError("the codes must have the shape of the input")
+    _need_contig(scale, "scale", torch.float32, (R,))
+    _check(fn(_ptr(src), R, K, src.stride(0) if R else K, _ptr(q), q.stride(0) if R else K, _ptr(scale),
+              _stream(stream, src.device)), what)
+    return q, scale
+
+
+def w8a8_quantize_act_fp8(x, xq=None, scale_a=None, stream=None):
+    """Per-token E4M3 quantization of bf16 x [M, K] -> (xq uint8 [M, K], scale_a fp32 [M])."""
+    return _quantize_fp8(_lib.w8a8_quantize_act_fp8, "w8a8_quantize_act_fp8", x, torch.bfloat16, xq, scale_a,
+                         stream)
+
+
+def w8a8_quantize_weight_fp8(w, wq=None, scale_w=None, stream=None):
+    """Per-output-channel E4M3 quantization of fp32 w [N, K] -> (wq uint8 [N, K], scale_w fp32 [N])."""
+    return _quantize_fp8(_lib.w8a8_quantize_weight_fp8, "w8a8_quantize_weight_fp8", w, torch.float32, wq,
+                         scale_w, stream)
+
+
+def _fp8_operands(xq, wq):
+    _need(xq, "xq", torch.uint8, 2)
+    _need(wq, "wq", torch.uint8, 2)
+    M, K = xq.shape
+    N, K2 = wq.shape
+    if K != K2:
+        raise ValueError(f"inner dimensions differ: xq has K={K}, wq has K={K2}")
+    _need_contig(xq, "xq", torch.uint8, (M, K))
+    _need_contig(wq, "wq", torch.uint8, (N, K))
+    return M, N, K
+
+
+def w8a8_gemm_fp8_ex(xq, wq, scale_a, scale_w, bias=None, out=None, config=None, stream=None):
+    """FP8 GEMM + dequant/bias epilogue, bf16 out [M, N]; config None = selected per shape."""
+    M, N, K = _fp8_operands(xq, wq)
+    _need_contig(scale_a, "scale_a", torch.float32, (M,))
+    _need_contig(scale_w, "scale_w", torch.float32, (N,))
+    if bias is not None:
+        _need_contig(bias, "bias", torch.bfloat16, (N,))
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    _need_contig(out, "out", torch.bfloat16, (M, N))
+    c = _cfg(config)
+    st = _lib.w8a8_gemm_fp8_ex(_ptr(xq), _ptr(wq), _ptr(scale_a), _ptr(scale_w), _ptr(bias), _ptr(out), M, N, K,
+                               ctypes.byref(c) if c is not None else None, _stream(stream, xq.device))
+    _check(st, "w8a8_gemm_fp8_ex")
+    return out
+
+
+def w8a8_gemm_fp8(xq, wq, scale_a, scale_w, bias=None, out=None, stream=None):
+    """out bf16 [M, N] = bf16((acc * scale_a[:, None]) * scale_w[None, :] + bias), acc the fp32 E4M3 product."""
+    return w8a8_gemm_fp8_ex(xq, wq, scale_a, scale_w, bias=bias, out=out, config=None, stream=stream)
+
+
+def w8a8_gemm_fp8_f32(xq, wq, acc=None, stream=None, config=None):
+    """Raw fp32 accumulators acc [M, N] of the E4M3 product xq @ wq^T."""
+    M, N, K = _fp8_operands(xq, wq)
+    if acc is None:
+        acc = torch.empty((M, N), dtype=torch.float32, device=xq.device)
+    _need_contig(acc, "acc", torch.float32, (M, N))
+    c = _cfg(config)
+    st = _lib.w8a8_gemm_fp8_f32_ex(_ptr(xq), _ptr(wq), _ptr(acc), M, N, K,
+                                   ctypes.byref(c) if c is not None else None, _stream(stream, xq.device))
+    _check(st, "w8a8_gemm_fp8_f32")
+    return acc
+
+
+def w8a8_gemm_fp8_f32_ex(xq, wq, acc=None, config=None, stream=None):
+    return w8a8_gemm_fp8_f32(xq, wq, acc=acc, stream=stream, config=config)
+
+
+def w8a8_linear_fp8(x, wq, scale_w, bias=None, out=None, ws_xq=None, ws_scale_a=None, stream=None):
+    """The FP8 linear layer: out bf16 [M, N] from bf16 x [M, K] and E4M3 wq uint8 [N, K]."""
+    _need(x, "x", torch.bfloat16, 2)
+    M, K = x.shape
+    _need(wq, "wq", torch.uint8, 2)
+    N = wq.shape[0]
+    if wq.shape[1] != K:
+        raise ValueError(f"inner dimensions differ: x has K={K}, wq has K={wq.shape[1]}")
+    _need_contig(x, "x", torch.bfloat16, (M, K))
+    _need_contig(wq, "wq", torch.uint8, (N, K))
+    _need_contig(scale_w, "scale_w", torch.float32, (N,))
+    if bias is not None:
+        _need_contig(bias, "bias", torch.bfloat16, (N,))
+    dev = x.device
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    if ws_xq is None:
+        ws_xq = torch.empty((M, K), dtype=torch.uint8, device=dev)
+    if ws_scale_a is None:
+        ws_scale_a = torch.empty((M,), dtype=torch.float32, device=dev)
+    _need_contig(out, "out", torch.bfloat16, (M, N))
+    _need_contig(ws_xq, "ws_xq", torch.uint8, (M, K))
+    _need_contig(ws_scale_a, "ws_scale_a", torch.float32, (M,))
+    _check(_lib.w8a8_linear_fp8(_ptr(x), _ptr(wq), _ptr(scale_w), _ptr(bias), _ptr(out), _ptr(ws_xq),
+                                _ptr(ws_scale_a), M, N, K, _stream(stream, dev)), "w8a8_linear_fp8")
     return out
 
 

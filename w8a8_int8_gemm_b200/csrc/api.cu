@@ -15,7 +15,7 @@
 namespace w8a8 {
 namespace {
 
-constexpr int64_t kMaxK = 133144;  // K * 127^2 < 2^31
+constexpr int64_t kMaxK = 133144;  // K * 127^2 < 2^31 (int8); the E4M3 path takes the same range
 constexpr int64_t kMaxMN = 2147483647;
 std::atomic<int64_t> g_timeout_ns{2000000000LL};
 
@@ -114,7 +114,7 @@ w8a8_status from_cuda(cudaError_t e) {
 w8a8_status gemm_common(const int8_t* xq, const int8_t* wq, const float* scale_a, const float* scale_w,
                         const void* bias, void* out, int64_t M, int64_t N, int64_t K,
                         const w8a8_gemm_config* user_cfg, GemmOut kind, cudaStream_t stream,
-                        bool overlap_prologue = false) {
+                        bool overlap_prologue = false, GemmElem elem = GemmElem::kInt8) {
   w8a8_status st = check_gemm_shape(M, N, K);
   if (st != W8A8_OK) return st;
   if (user_cfg != nullptr && (st = check_config(*user_cfg)) != W8A8_OK) return st;
@@ -139,6 +139,7 @@ w8a8_status gemm_common(const int8_t* xq, const int8_t* wq, const float* scale_a
   a.N = N;
   a.K = K;
   a.out_kind = kind;
+  a.elem = elem;
   a.timeout_ns = static_cast<uint64_t>(g_timeout_ns.load());
   a.overlap_prologue = overlap_prologue;
   GemmConfig c{cfg.block_m, cfg.block_n, cfg.stages, cfg.grid, cfg.raster_group};
@@ -146,7 +147,7 @@ w8a8_status gemm_common(const int8_t* xq, const int8_t* wq, const float* scale_a
 }
 
 w8a8_status quantize_common(bool act, const void* x, int64_t M, int64_t K, int64_t ldx, int8_t* xq, int64_t ldxq,
-                            float* scale, cudaStream_t stream) {
+                            float* scale, cudaStream_t stream, bool e4m3 = false) {
   if (M < 0 || M > kMaxMN || K < 16 || K > kMaxK || K % 16 != 0) return W8A8_ERR_INVALID_ARG;
   if (ldx < K || ldxq < K) return W8A8_ERR_INVALID_ARG;
   if (M == 0) return W8A8_OK;
@@ -157,9 +158,16 @@ w8a8_status quantize_common(bool act, const void* x, int64_t M, int64_t K, int64
   DeviceInfo dev;
   w8a8_status st = current_device(&dev);
   if (st != W8A8_OK) return st;
-  const cudaError_t e = act ? launch_quantize_act(x, M, K, ldx, xq, ldxq, scale, stream)
-                            : launch_quantize_weight(static_cast<const float*>(x), M, K, ldx, xq, ldxq, scale,
-                                                     stream);
+  const float* w = static_cast<const float*>(x);
+  uint8_t* codes = reinterpret_cast<uint8_t*>(xq);
+  cudaError_t e;
+  if (e4m3) {
+    e = act ? launch_quantize_act_e4m3(x, M, K, ldx, codes, ldxq, scale, stream)
+            : launch_quantize_weight_e4m3(w, M, K, ldx, codes, ldxq, scale, stream);
+  } else {
+    e = act ? launch_quantize_act(x, M, K, ldx, xq, ldxq, scale, stream)
+            : launch_quantize_weight(w, M, K, ldx, xq, ldxq, scale, stream);
+  }
   return from_cuda(e);
 }
 
@@ -211,13 +219,13 @@ w8a8_status w8a8_gemm_ex(const int8_t* xq, const int8_t* wq, const float* scale_
 
 w8a8_status w8a8_gemm_i32(const int8_t* xq, const int8_t* wq, int32_t* acc, int64_t M, int64_t N, int64_t K,
                           w8a8_stream_t stream) {
-  return gemm_common(xq, wq, nullptr, nullptr, nullptr, acc, M, N, K, nullptr, GemmOut::kInt32,
+  return gemm_common(xq, wq, nullptr, nullptr, nullptr, acc, M, N, K, nullptr, GemmOut::kAcc32,
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 w8a8_status w8a8_gemm_i32_ex(const int8_t* xq, const int8_t* wq, int32_t* acc, int64_t M, int64_t N, int64_t K,
                              const w8a8_gemm_config* cfg, w8a8_stream_t stream) {
-  return gemm_common(xq, wq, nullptr, nullptr, nullptr, acc, M, N, K, cfg, GemmOut::kInt32,
+  return gemm_common(xq, wq, nullptr, nullptr, nullptr, acc, M, N, K, cfg, GemmOut::kAcc32,
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -276,6 +284,66 @@ w8a8_status w8a8_linear_fused(const void* x, const int8_t* wq, const float* scal
   a.sync = ws_sync;
   GemmConfig c{cfg.block_m, cfg.block_n, cfg.stages, cfg.grid, cfg.raster_group};
   return from_cuda(launch_gemm(a, c, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// ------------------------------------------------------------ E4M3 variant
+
+w8a8_status w8a8_quantize_act_fp8(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* xq, int64_t ldxq,
+                                  float* scale_a, w8a8_stream_t stream) {
+  return quantize_common(true, x, M, K, ldx, reinterpret_cast<int8_t*>(xq), ldxq, scale_a,
+                         reinterpret_cast<cudaStream_t>(stream), /*e4m3=*/true);
+}
+
+w8a8_status w8a8_quantize_weight_fp8(const float* w, int64_t N, int64_t K, int64_t ldw, uint8_t* wq, int64_t ldwq,
+                                     float* scale_w, w8a8_stream_t stream) {
+  return quantize_common(false, w, N, K, ldw, reinterpret_cast<int8_t*>(wq), ldwq, scale_w,
+                         reinterpret_cast<cudaStream_t>(stream), /*e4m3=*/true);
+}
+
+w8a8_status w8a8_gemm_fp8_ex(const uint8_t* xq, const uint8_t* wq, const float* scale_a, const float* scale_w,
+                             const void* bias, void* out, int64_t M, int64_t N, int64_t K,
+                             const w8a8_gemm_config* cfg, w8a8_stream_t stream) {
+  return gemm_common(reinterpret_cast<const int8_t*>(xq), reinterpret_cast<const int8_t*>(wq), scale_a, scale_w,
+                     bias, out, M, N, K, cfg, GemmOut::kBf16Dequant, reinterpret_cast<cudaStream_t>(stream),
+                     /*overlap_prologue=*/false, GemmElem::kE4M3);
+}
+
+w8a8_status w8a8_gemm_fp8(const uint8_t* xq, const uint8_t* wq, const float* scale_a, const float* scale_w,
+                          const void* bias, void* out, int64_t M, int64_t N, int64_t K, w8a8_stream_t stream) {
+  return w8a8_gemm_fp8_ex(xq, wq, scale_a, scale_w, bias, out, M, N, K, nullptr, stream);
+}
+
+w8a8_status w8a8_gemm_fp8_f32_ex(const uint8_t* xq, const uint8_t* wq, float* acc, int64_t M, int64_t N, int64_t K,
+                                 const w8a8_gemm_config* cfg, w8a8_stream_t stream) {
+  return gemm_common(reinterpret_cast<const int8_t*>(xq), reinterpret_cast<const int8_t*>(wq), nullptr, nullptr,
+                     nullptr, acc, M, N, K, cfg, GemmOut::kAcc32, reinterpret_cast<cudaStream_t>(stream),
+                     /*overlap_prologue=*/false, GemmElem::kE4M3);
+}
+
+w8a8_status w8a8_gemm_fp8_f32(const uint8_t* xq, const uint8_t* wq, float* acc, int64_t M, int64_t N, int64_t K,
+                              w8a8_stream_t stream) {
+  return w8a8_gemm_fp8_f32_ex(xq, wq, acc, M, N, K, nullptr, stream);
+}
+
+w8a8_status w8a8_linear_fp8(const void* x, const uint8_t* wq, const float* scale_w, const void* bias, void* out,
+                            uint8_t* ws_xq, float* ws_scale_a, int64_t M, int64_t N, int64_t K,
+                            w8a8_stream_t stream) {
+  w8a8_status st = check_gemm_shape(M, N, K);
+  if (st != W8A8_OK) return st;
+  if (M == 0 || N == 0) return W8A8_OK;
+  if (x == nullptr || wq == nullptr || scale_w == nullptr || out == nullptr || ws_xq == nullptr ||
+      ws_scale_a == nullptr) {
+    return W8A8_ERR_INVALID_ARG;
+  }
+  if (!aligned16(x) || !aligned16(wq) || !aligned16(scale_w) || !aligned16(bias) || !aligned16(out) ||
+      !aligned16(ws_xq) || !aligned16(ws_scale_a)) {
+    return W8A8_ERR_ALIGNMENT;
+  }
+  st = w8a8_quantize_act_fp8(x, M, K, K, ws_xq, K, ws_scale_a, stream);
+  if (st != W8A8_OK) return st;
+  return gemm_common(reinterpret_cast<const int8_t*>(ws_xq), reinterpret_cast<const int8_t*>(wq), ws_scale_a,
+                     scale_w, bias, out, M, N, K, nullptr, GemmOut::kBf16Dequant,
+                     reinterpret_cast<cudaStream_t>(stream), /*overlap_prologue=*/true, GemmElem::kE4M3);
 }
 
 int64_t w8a8_linear_sync_words(int64_t M) { return M < 0 ? 0 : linear_sync_words(M); }

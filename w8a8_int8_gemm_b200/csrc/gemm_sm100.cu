@@ -27,6 +27,11 @@
 //   * the accumulator is double-buffered in tensor memory (2 x BLOCK_N
 //     columns), so the epilogue of one tile overlaps the MMAs of the next.
 //
+// The same kernel runs the FP8 variant (OCP E4M3 operands, the paper's
+// comparison baseline): tcgen05.mma.kind::f8f6f4, also K=32 bytes per
+// instruction, so the tiles, the ring and the swizzle are unchanged; the
+// accumulators are fp32 and the epilogue uses them as they are.
+//
 // Every mbarrier wait is bounded in time (see sm100_ptx.cuh); on timeout the
 // kernel records the site in the device error word, lets its in-flight
 // copies and MMAs finish (again bounded), frees tensor memory and exits.
@@ -124,7 +129,9 @@ __device__ __forceinline__ void tile_coords(int tile, const Params& p, int& mb, 
 
 // Dequantize 32 accumulators of one row into 16 packed bf16 pairs:
 // y = (fl32(acc) * sa) * sw[n] + bias[n], each op rounded, with sw / bias
-// (32 columns) read from shared memory.
+// (32 columns) read from shared memory.  kF32Acc: the accumulators are
+// already fp32 (E4M3 operands); otherwise int32, converted with rounding.
+template <bool kF32Acc>
 __device__ __forceinline__ void dequant_32(const uint32_t (&v)[32], float sa, const float* sw_s,
                                            const uint16_t* bias_s, uint32_t* packed) {
 #pragma unroll
@@ -140,7 +147,8 @@ __device__ __forceinline__ void dequant_32(const uint32_t (&v)[32], float sa, co
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const float b = __uint_as_float(j ? (w[i] & 0xFFFF0000u) : (w[i] << 16));
-        float t = __int2float_rn(static_cast<int>(v[8 * g + 2 * i + j]));
+        const uint32_t a = v[8 * g + 2 * i + j];
+        float t = kF32Acc ? __uint_as_float(a) : __int2float_rn(static_cast<int>(a));
         t = __fmul_rn(t, sa);
         t = __fmul_rn(t, sw[2 * i + j]);
         y[j] = __fadd_rn(t, b);
@@ -169,7 +177,7 @@ __device__ __forceinline__ void dequant_32(const uint32_t (&v)[32], float sa, co
 // A, and the epilogue before reading its scales.  All CTAs are co-resident
 // (cooperative launch), so these waits cannot deadlock; they are bounded
 // all the same.  The last CTA to finish resets the counters to zero.
-template <int BN, GemmOut OUT, bool PAIR, bool FUSE>
+template <int BN, GemmOut OUT, bool PAIR, bool FUSE, GemmElem EL>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_b_half, const __grid_constant__ CUtensorMap tm_d,
@@ -180,8 +188,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kB = kBRows * kBlockK;
   constexpr uint32_t kTxBytes = (PAIR ? 2 : 1) * (kA + kB);
   constexpr uint32_t kTmemCols = 2 * BN;  // two accumulator buffers; 256 or 512 (power of two)
-  constexpr uint32_t kIdesc = make_idesc_i8(kTileM, BN);
-  constexpr uint32_t kIdescHalf = make_idesc_i8(kTileM, BN / 2);  // half-width tail items
+  constexpr bool kE4M3 = EL == GemmElem::kE4M3;
+  constexpr uint32_t kIdesc = kE4M3 ? make_idesc_e4m3(kTileM, BN) : make_idesc_i8(kTileM, BN);
+  // half-width tail items
+  constexpr uint32_t kIdescHalf = kE4M3 ? make_idesc_e4m3(kTileM, BN / 2) : make_idesc_i8(kTileM, BN / 2);
   constexpr int kEpiArrivals = (PAIR ? 2 : 1) * kEpiWarps;
 
   extern __shared__ uint8_t smem_raw[];
@@ -350,8 +360,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               // Advance the start address by 32 bytes (2 in units of 16 B)
               // per K=32 slice inside the 128-byte swizzled row.
               const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-              if constexpr (PAIR) {
+              if constexpr (PAIR && kE4M3) {
+                mma_e4m3_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, acc);
+              } else if constexpr (PAIR) {
                 mma_i8_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, acc);
+              } else if constexpr (kE4M3) {
+                mma_e4m3(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, acc);
               } else {
                 mma_i8(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, acc);
               }
@@ -512,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if constexpr (OUT == GemmOut::kBf16Dequant) {
           uint32_t pk[16];
-          dequant_32(cur, sa, ps_w + cl, ps_b + cl, pk);
+          dequant_32<kE4M3>(cur, sa, ps_w + cl, ps_b + cl, pk);
           if (in_range) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -643,9 +657,10 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem, const void
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, GemmOut OUT, bool PAIR, bool FUSE>
+template <int BN, GemmOut OUT, bool PAIR, bool FUSE, GemmElem EL = GemmElem::kInt8>
 cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t stream) {
   static_assert(!(FUSE && PAIR), "the fused linear layer runs on single CTAs");
+  static_assert(!(FUSE && EL == GemmElem::kE4M3), "the fused linear layer is int8 only");
   constexpr int kTileM = PAIR ? 2 * kBlockM : kBlockM;
   constexpr int kBRows = PAIR ? BN / 2 : BN;
   CUtensorMap tm_a, tm_b, tm_b_half, tm_d;
@@ -659,7 +674,8 @@ cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t 
   if constexpr (OUT == GemmOut::kBf16Dequant) {
     ok = ok && encode_2d(&tm_d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.out, a.M, a.N, 32, 64);
   } else {
-    ok = ok && encode_2d(&tm_d, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, a.out, a.M, a.N, 32, 32);
+    ok = ok && encode_2d(&tm_d, EL == GemmElem::kE4M3 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_INT32,
+                         4, a.out, a.M, a.N, 32, 32);
   }
   if (!ok) return cudaErrorInvalidValue;
 
@@ -689,7 +705,7 @@ cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t 
   if (e != cudaSuccess) return e;
 
   const int smem = smem_bytes(PAIR, BN, cfg.stages);
-  auto kernel = gemm_w8a8_kernel<BN, OUT, PAIR, FUSE>;
+  auto kernel = gemm_w8a8_kernel<BN, OUT, PAIR, FUSE, EL>;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   // Persistent grid: one CTA (or CTA pair) per tile at most.
@@ -759,35 +775,45 @@ int gemm_max_stages(int block_m, int block_n) {
   return s;
 }
 
+// Non-fused launches of one operand format.
+template <GemmElem EL>
+cudaError_t launch_plain(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t stream) {
+  using O = GemmOut;
+  const bool bf16 = a.out_kind == O::kBf16Dequant;
+  if (cfg.block_m == 256) {
+    if (cfg.block_n == 256) {
+      return bf16 ? launch_typed<256, O::kBf16Dequant, true, false, EL>(a, cfg, stream)
+                  : launch_typed<256, O::kAcc32, true, false, EL>(a, cfg, stream);
+    }
+    if (cfg.block_n == 128) {
+      return bf16 ? launch_typed<128, O::kBf16Dequant, true, false, EL>(a, cfg, stream)
+                  : launch_typed<128, O::kAcc32, true, false, EL>(a, cfg, stream);
+    }
+  } else if (cfg.block_m == 128) {
+    if (cfg.block_n == 256) {
+      return bf16 ? launch_typed<256, O::kBf16Dequant, false, false, EL>(a, cfg, stream)
+                  : launch_typed<256, O::kAcc32, false, false, EL>(a, cfg, stream);
+    }
+    if (cfg.block_n == 128) {
+      return bf16 ? launch_typed<128, O::kBf16Dequant, false, false, EL>(a, cfg, stream)
+                  : launch_typed<128, O::kAcc32, false, false, EL>(a, cfg, stream);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_gemm(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t stream) {
-  const bool bf16 = a.out_kind == GemmOut::kBf16Dequant;
   using O = GemmOut;
   if (a.fused) {
-    if (!bf16 || cfg.block_m != 128) return cudaErrorInvalidValue;
+    if (a.out_kind != O::kBf16Dequant || a.elem != GemmElem::kInt8 || cfg.block_m != 128) {
+      return cudaErrorInvalidValue;
+    }
     if (cfg.block_n == 256) return launch_typed<256, O::kBf16Dequant, false, true>(a, cfg, stream);
     if (cfg.block_n == 128) return launch_typed<128, O::kBf16Dequant, false, true>(a, cfg, stream);
     return cudaErrorInvalidValue;
   }
-  if (cfg.block_m == 256) {
-    if (cfg.block_n == 256) {
-      return bf16 ? launch_typed<256, O::kBf16Dequant, true, false>(a, cfg, stream)
-                  : launch_typed<256, O::kInt32, true, false>(a, cfg, stream);
-    }
-    if (cfg.block_n == 128) {
-      return bf16 ? launch_typed<128, O::kBf16Dequant, true, false>(a, cfg, stream)
-                  : launch_typed<128, O::kInt32, true, false>(a, cfg, stream);
-    }
-  } else if (cfg.block_m == 128) {
-    if (cfg.block_n == 256) {
-      return bf16 ? launch_typed<256, O::kBf16Dequant, false, false>(a, cfg, stream)
-                  : launch_typed<256, O::kInt32, false, false>(a, cfg, stream);
-    }
-    if (cfg.block_n == 128) {
-      return bf16 ? launch_typed<128, O::kBf16Dequant, false, false>(a, cfg, stream)
-                  : launch_typed<128, O::kInt32, false, false>(a, cfg, stream);
-    }
-  }
-  return cudaErrorInvalidValue;
+  return a.elem == GemmElem::kE4M3 ? launch_plain<GemmElem::kE4M3>(a, cfg, stream)
+                                   : launch_plain<GemmElem::kInt8>(a, cfg, stream);
 }
 
 cudaError_t launch_selftest_wait(uint64_t timeout_ns, cudaStream_t stream) {

@@ -16,10 +16,16 @@ struct GemmConfig {
   int raster_group;
 };
 
-enum class GemmOut { kBf16Dequant = 0, kInt32 = 1 };
+// kAcc32: the raw 32-bit accumulators (int32 for int8 operands, fp32 for
+// E4M3 operands) instead of the dequantized bf16 output.
+enum class GemmOut { kBf16Dequant = 0, kAcc32 = 1 };
+
+// Operand format: int8 (tcgen05 kind::i8, int32 accumulators) or OCP E4M3
+// (kind::f8f6f4, fp32 accumulators).
+enum class GemmElem { kInt8 = 0, kE4M3 = 1 };
 
 struct GemmArgs {
-  const int8_t* xq;
+  const int8_t* xq;  // int8 or E4M3 codes (bytes)
   const int8_t* wq;
   const float* scale_a;
   const float* scale_w;
@@ -27,6 +33,7 @@ struct GemmArgs {
   void* out;         // bf16 [M, N] or int32 [M, N]
   int64_t M, N, K;
   GemmOut out_kind;
+  GemmElem elem = GemmElem::kInt8;
   uint64_t timeout_ns;
   // The fused linear layer: quantize x [M, K] (bf16, row stride ldx) into
   // xq / scale_a inside the GEMM kernel (xq and scale_a are then outputs);
@@ -48,6 +55,10 @@ cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int64_t ldx
                                 float* scale, cudaStream_t stream);
 cudaError_t launch_quantize_weight(const float* w, int64_t N, int64_t K, int64_t ldw, int8_t* q, int64_t ldq,
                                    float* scale, cudaStream_t stream);
+cudaError_t launch_quantize_act_e4m3(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, int64_t ldq,
+                                     float* scale, cudaStream_t stream);
+cudaError_t launch_quantize_weight_e4m3(const float* w, int64_t N, int64_t K, int64_t ldw, uint8_t* q, int64_t ldq,
+                                        float* scale, cudaStream_t stream);
 
 // Largest stage count the shared memory holds for a tile shape (0 if none).
 // block_m 128: one CTA per tile; block_m 256: a CTA pair (cluster of 2).

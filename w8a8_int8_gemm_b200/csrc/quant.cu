@@ -32,6 +32,16 @@
 // with IEEE division (__fdiv_rn) in an out-of-line path.  Rows whose scale is
 // not a normal number, or whose reciprocal is not finite, take the division
 // for every element.
+//
+// FP8 variant (OCP E4M3 codes; B200's native FP8 path, the comparison
+// baseline of the same paper): the same scheme with 448, the largest finite
+// E4M3 value, in place of 127:
+//   scale[r] = fl32(max_k |x[r,k]| / 448)
+//   q[r,k]   = e4m3_rne(clamp(fl32(x[r,k] / scale[r]), -448, 448)), 0 if scale[r] == 0
+// Each element takes one IEEE division and one hardware conversion
+// (cvt.rn.satfinite.e4m3x2.f32: round to nearest even, saturating), which is
+// the definition term by term; a negative quotient that rounds to zero keeps
+// its sign (code 0x80).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -47,21 +57,21 @@ namespace {
 // Rows of up to 32 * VPL vectors: the whole row in registers.  Seven
 // 128-thread blocks per SM (at most 72 registers) keep 28 rows per SM in
 // flight, so a 4096-token batch is resident in one wave on 148 SMs.
-template <typename T, int VPL>
-__global__ void __launch_bounds__(128, (VPL <= 12 ? 7 : 5)) quantize_rows_regs_kernel(const T* __restrict__ x, int64_t M, int64_t K,
-                                                                 int64_t ldx, int8_t* __restrict__ q, int64_t ldq,
-                                                                 float* __restrict__ scale) {
+template <typename T, int VPL, qrow::Code C>
+__global__ void __launch_bounds__(128, (VPL <= 12 ? 7 : 5))
+    quantize_rows_regs_kernel(const T* __restrict__ x, int64_t M, int64_t K, int64_t ldx, int8_t* __restrict__ q,
+                              int64_t ldq, float* __restrict__ scale) {
   pdl_launch_dependents();  // a GEMM launched after this may be scheduled already
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= M) return;
-  const float s = qrow::quantize_row<T, VPL>(reinterpret_cast<const uint4*>(x + row * ldx),
-                                             static_cast<int>(K / qrow::Vec<T>::kElems), q + row * ldq, lane);
+  const float s = qrow::quantize_row<T, VPL, C>(reinterpret_cast<const uint4*>(x + row * ldx),
+                                                static_cast<int>(K / qrow::Vec<T>::kElems), q + row * ldq, lane);
   if (lane == 0) scale[row] = s;
 }
 
 // Any row length: absmax pass, then a second pass that reads the row again.
-template <typename T>
+template <typename T, qrow::Code C>
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict__ x, int64_t M, int64_t K,
                                                             int64_t ldx, int8_t* __restrict__ q, int64_t ldq,
                                                             float* __restrict__ scale) {
@@ -69,36 +79,36 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict_
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= M) return;
-  const float s = qrow::quantize_row<T, 0>(reinterpret_cast<const uint4*>(x + row * ldx),
-                                           static_cast<int>(K / qrow::Vec<T>::kElems), q + row * ldq, lane);
+  const float s = qrow::quantize_row<T, 0, C>(reinterpret_cast<const uint4*>(x + row * ldx),
+                                              static_cast<int>(K / qrow::Vec<T>::kElems), q + row * ldq, lane);
   if (lane == 0) scale[row] = s;
 }
 
-template <typename T, int VPL>
+template <typename T, int VPL, qrow::Code C>
 void launch_regs(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq, float* scale,
                  cudaStream_t stream) {
   const int threads = 128;
   const int64_t blocks = (M + (threads / 32) - 1) / (threads / 32);
-  quantize_rows_regs_kernel<T, VPL>
+  quantize_rows_regs_kernel<T, VPL, C>
       <<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, M, K, ldx, q, ldq, scale);
 }
 
-template <typename T>
+template <typename T, qrow::Code C>
 cudaError_t launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq, float* scale,
                             cudaStream_t stream) {
   const int64_t per_lane = (K / qrow::Vec<T>::kElems + 31) / 32;
   if (per_lane <= 4) {
-    launch_regs<T, 4>(x, M, K, ldx, q, ldq, scale, stream);
+    launch_regs<T, 4, C>(x, M, K, ldx, q, ldq, scale, stream);
   } else if (per_lane <= 8) {
-    launch_regs<T, 8>(x, M, K, ldx, q, ldq, scale, stream);
+    launch_regs<T, 8, C>(x, M, K, ldx, q, ldq, scale, stream);
   } else if (per_lane <= 12) {
-    launch_regs<T, 12>(x, M, K, ldx, q, ldq, scale, stream);
+    launch_regs<T, 12, C>(x, M, K, ldx, q, ldq, scale, stream);
   } else if (per_lane <= 16) {
-    launch_regs<T, 16>(x, M, K, ldx, q, ldq, scale, stream);
+    launch_regs<T, 16, C>(x, M, K, ldx, q, ldq, scale, stream);
   } else {
     const int threads = 256;
     const int64_t blocks = (M + (threads / 32) - 1) / (threads / 32);
-    quantize_rows_kernel<T><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, M, K, ldx, q, ldq, scale);
+    quantize_rows_kernel<T, C><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, M, K, ldx, q, ldq, scale);
   }
   return cudaGetLastError();
 }
@@ -107,12 +117,24 @@ cudaError_t launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_
 
 cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq,
                                 float* scale, cudaStream_t stream) {
-  return launch_quantize<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x), M, K, ldx, q, ldq, scale, stream);
+  return launch_quantize<__nv_bfloat16, qrow::Code::kInt8>(static_cast<const __nv_bfloat16*>(x), M, K, ldx, q, ldq,
+                                                           scale, stream);
 }
 
 cudaError_t launch_quantize_weight(const float* w, int64_t N, int64_t K, int64_t ldw, int8_t* q, int64_t ldq,
                                    float* scale, cudaStream_t stream) {
-  return launch_quantize<float>(w, N, K, ldw, q, ldq, scale, stream);
+  return launch_quantize<float, qrow::Code::kInt8>(w, N, K, ldw, q, ldq, scale, stream);
+}
+
+cudaError_t launch_quantize_act_e4m3(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, int64_t ldq,
+                                     float* scale, cudaStream_t stream) {
+  return launch_quantize<__nv_bfloat16, qrow::Code::kE4M3>(static_cast<const __nv_bfloat16*>(x), M, K, ldx,
+                                                           reinterpret_cast<int8_t*>(q), ldq, scale, stream);
+}
+
+cudaError_t launch_quantize_weight_e4m3(const float* w, int64_t N, int64_t K, int64_t ldw, uint8_t* q, int64_t ldq,
+                                        float* scale, cudaStream_t stream) {
+  return launch_quantize<float, qrow::Code::kE4M3>(w, N, K, ldw, reinterpret_cast<int8_t*>(q), ldq, scale, stream);
 }
 
 }  // namespace w8a8

@@ -1,17 +1,28 @@
-// quant_row.cuh -- one warp quantizes one row (symmetric absmax, int8).
+// quant_row.cuh -- one warp quantizes one row (symmetric absmax, int8 or
+// OCP E4M3 codes).
 //
 // Shared by the standalone row quantizers (quant.cu) and the fused linear
 // kernel (gemm_sm100.cu), which quantizes activation rows inside the GEMM.
-// The rule, and why the product shortcut decides the same codes as the
-// IEEE division, are stated at the top of quant.cu.
+// The rules, and why the int8 product shortcut decides the same codes as
+// the IEEE division, are stated at the top of quant.cu.
 #pragma once
 
 #include <cuda_bf16.h>
 
 #include <cstdint>
 
+#include "sm100_ptx.cuh"
+
 namespace w8a8 {
 namespace qrow {
+
+// Code format: int8 (scale absmax / 127) or E4M3 (scale absmax / 448).
+enum class Code { kInt8, kE4M3 };
+
+template <Code C>
+__device__ __forceinline__ constexpr float code_max() {
+  return C == Code::kInt8 ? 127.0f : 448.0f;
+}
 
 template <typename T>
 struct Vec;
@@ -125,20 +136,53 @@ __device__ __forceinline__ void quantize_vec(const uint4& v, float s, float r, b
   quantize_vec_div<T>(v, s, dst);
 }
 
+// E4M3 codes of one vector: e4m3_rne(clamp(fl32(x / s), -448, 448)), one
+// IEEE division per element and one rounding to E4M3 (the clamp is explicit
+// although the conversion saturates: the definition clamps).
+template <typename T>
+__device__ __forceinline__ void quantize_vec_e4m3(const uint4& v, float s, int8_t* dst) {
+  constexpr int E = Vec<T>::kElems;
+  float f[E];
+  Vec<T>::unpack(v, f);
+  uint32_t h[E / 2];
+#pragma unroll
+  for (int i = 0; i < E / 2; ++i) {
+    const float a = fminf(fmaxf(__fdiv_rn(f[2 * i], s), -448.0f), 448.0f);
+    const float b = fminf(fmaxf(__fdiv_rn(f[2 * i + 1], s), -448.0f), 448.0f);
+    h[i] = cvt_e4m3x2(a, b);
+  }
+  if constexpr (E == 8) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = h[0] | (h[1] << 16);
+  }
+}
+
 struct RowScale {
   float s, r;
   bool zero, fast;
 };
 
+template <Code C = Code::kInt8>
 __device__ __forceinline__ RowScale row_scale(float amax) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   RowScale rs;
-  rs.s = __fdiv_rn(amax, 127.0f);
+  rs.s = __fdiv_rn(amax, code_max<C>());
   rs.zero = (rs.s == 0.0f);  // all-zero row (or an fp32 row whose scale underflows): codes 0
   rs.r = rs.zero ? 0.0f : __frcp_rn(rs.s);
   rs.fast = !rs.zero && rs.s >= 1.17549435e-38f && isfinite(rs.r);
   return rs;
+}
+
+// Codes of one vector of a row whose scale is nonzero.
+template <typename T, Code C>
+__device__ __forceinline__ void encode_vec(const uint4& v, const RowScale& rs, int8_t* dst) {
+  if constexpr (C == Code::kInt8) {
+    quantize_vec<T>(v, rs.s, rs.r, rs.fast, dst);
+  } else {
+    quantize_vec_e4m3<T>(v, rs.s, dst);
+  }
 }
 
 template <int E>
@@ -154,7 +198,7 @@ __device__ __forceinline__ void store_zero(int8_t* dst) {
 // the row's scale in every lane.  VPL > 0: rows of up to 32 * VPL vectors,
 // all loads issued at once and the row kept in registers; VPL == 0: any
 // length, an absmax pass and a second pass that reads the row again.
-template <typename T, int VPL>
+template <typename T, int VPL, Code C = Code::kInt8>
 __device__ __forceinline__ float quantize_row(const uint4* __restrict__ xr, int nvec, int8_t* __restrict__ qr,
                                               int lane) {
   constexpr int E = Vec<T>::kElems;
@@ -168,7 +212,7 @@ __device__ __forceinline__ float quantize_row(const uint4* __restrict__ xr, int 
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) amax = fmaxf(amax, vec_absmax<T>(c[i]));
-    const RowScale rs = row_scale(amax);
+    const RowScale rs = row_scale<C>(amax);
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int v = lane + 32 * i;
@@ -176,7 +220,7 @@ __device__ __forceinline__ float quantize_row(const uint4* __restrict__ xr, int 
         if (rs.zero) {
           store_zero<E>(qr + E * v);
         } else {
-          quantize_vec<T>(c[i], rs.s, rs.r, rs.fast, qr + E * v);
+          encode_vec<T, C>(c[i], rs, qr + E * v);
         }
       }
     }
@@ -193,7 +237,7 @@ __device__ __forceinline__ float quantize_row(const uint4* __restrict__ xr, int 
       for (int i = 0; i < 8; ++i) amax = fmaxf(amax, vec_absmax<T>(a[i]));
     }
     for (; v < nvec; v += 32) amax = fmaxf(amax, vec_absmax<T>(__ldg(xr + v)));
-    const RowScale rs = row_scale(amax);
+    const RowScale rs = row_scale<C>(amax);
     // pass 2: codes
     v = lane;
     for (; v + 96 < nvec; v += 128) {
@@ -205,7 +249,7 @@ __device__ __forceinline__ float quantize_row(const uint4* __restrict__ xr, int 
         if (rs.zero) {
           store_zero<E>(qr + E * (v + 32 * i));
         } else {
-          quantize_vec<T>(a[i], rs.s, rs.r, rs.fast, qr + E * (v + 32 * i));
+          encode_vec<T, C>(a[i], rs, qr + E * (v + 32 * i));
         }
       }
     }
@@ -213,7 +257,7 @@ __device__ __forceinline__ float quantize_row(const uint4* __restrict__ xr, int 
       if (rs.zero) {
         store_zero<E>(qr + E * v);
       } else {
-        quantize_vec<T>(__ldg(xr + v), rs.s, rs.r, rs.fast, qr + E * v);
+        encode_vec<T, C>(__ldg(xr + v), rs, qr + E * v);
       }
     }
     return rs.s;
