@@ -178,10 +178,23 @@ def test_acc_every_config(w8, cfg):
     assert np.array_equal(_acc(w8, xq, wq, config=cfg), oracle.gemm_fp8(xq, wq))
 
 
-@pytest.mark.parametrize("shape,grid", [((300, 776, 656), 5), ((129, 520, 1040), 4)], ids=lambda v: str(v))
-def test_acc_tail_halves(w8, shape, grid):
+@pytest.mark.parametrize("K,stages", [(384, 6), (1024, 4), (2048, 5)])
+def test_acc_pair_double_chunk_stages(w8, K, stages):
+    """CTA pairs loading two K-chunks per box (K % 128 == 0, ring >= 4 chunks)."""
+    rng = np.random.default_rng(K + stages)
+    M, N = 300, 520
+    xq, wq = _exact_codes(rng, M, K), _exact_codes(rng, N, K)
+    for bn in (256, 128):
+        cfg = dict(block_m=256, block_n=bn, stages=stages, grid=148, raster_group=8)
+        assert np.array_equal(_acc(w8, xq, wq, config=cfg), oracle.gemm_fp8(xq, wq)), cfg
+
+
+@pytest.mark.parametrize("shape,grid,bm,stages", [((300, 776, 656), 5, 128, 4), ((129, 520, 1040), 4, 128, 4),
+                                                  ((300, 776, 1024), 12, 256, 6), ((520, 1032, 640), 24, 256, 5)],
+                         ids=lambda v: str(v))
+def test_acc_tail_halves(w8, shape, grid, bm, stages):
     M, N, K = shape
-    cfg = dict(block_m=128, block_n=256, stages=4, grid=grid, raster_group=1)
+    cfg = dict(block_m=bm, block_n=256, stages=stages, grid=grid, raster_group=1)
     rng = np.random.default_rng(M + grid)
     xq, wq = _exact_codes(rng, M, K), _exact_codes(rng, N, K)
     assert np.array_equal(_acc(w8, xq, wq, config=cfg), oracle.gemm_fp8(xq, wq))

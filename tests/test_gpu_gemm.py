@@ -65,6 +65,47 @@ def test_i32_every_config(w8, cfg):
     assert np.array_equal(_i32(w8, xq, wq, config=cfg), oracle.gemm_i64(xq, wq))
 
 
+# CTA pairs with K a multiple of 128 and at least 4 chunks of ring depth load
+# boxes spanning two K-chunks; K = 128 (mod 256) leaves the second chunk of
+# the last stage outside the tensor (filled with zeros).
+PAIR_CHUNK_CASES = [((300, 776, 128), 6), ((300, 776, 384), 6), ((257, 520, 1024), 4), ((129, 264, 3072), 5),
+                    ((520, 1032, 640), 8)]
+
+
+@pytest.mark.parametrize("shape,stages", PAIR_CHUNK_CASES, ids=lambda v: str(v))
+@pytest.mark.parametrize("bn", [256, 128])
+def test_pair_double_chunk_stages(w8, shape, stages, bn):
+    M, N, K = shape
+    if stages > (6 if bn == 256 else 8):
+        pytest.skip("ring deeper than shared memory holds for this tile")
+    rng = np.random.default_rng(M + K + bn)
+    xq, wq = _codes(rng, M, K), _codes(rng, N, K)
+    for grid, rg in ((148, 8), (4, 1)):
+        cfg = dict(block_m=256, block_n=bn, stages=stages, grid=grid, raster_group=rg)
+        assert np.array_equal(_i32(w8, xq, wq, config=cfg), oracle.gemm_i64(xq, wq)), cfg
+    got, want = _bf16_gemm_case(w8, M, N, K, M * 5 + K, True,
+                                dict(block_m=256, block_n=bn, stages=stages, grid=148, raster_group=8))
+    assert bf16_ulp_diff(got, want).max() <= 1
+
+
+# CTA-pair grids with a short last round (256 x 256 tiles; its tiles run as
+# 256 x 128 items): 8 tiles on 6 pairs, 15 tiles on 12 pairs, with single-
+# (K % 128 != 0) and double-chunk stages.
+PAIR_TAIL_CASES = [((300, 776, 656), 12, 6), ((300, 776, 1024), 12, 6), ((520, 1032, 640), 24, 6),
+                   ((520, 1032, 640), 24, 4), ((520, 1032, 3072), 24, 5)]
+
+
+@pytest.mark.parametrize("shape,grid,stages", PAIR_TAIL_CASES, ids=lambda v: str(v))
+def test_pair_tail_halves(w8, shape, grid, stages):
+    M, N, K = shape
+    cfg = dict(block_m=256, block_n=256, stages=stages, grid=grid, raster_group=1)
+    rng = np.random.default_rng(M + grid + K)
+    xq, wq = _codes(rng, M, K), _codes(rng, N, K)
+    assert np.array_equal(_i32(w8, xq, wq, config=cfg), oracle.gemm_i64(xq, wq))
+    got, want = _bf16_gemm_case(w8, M, N, K, M * 7 + grid + K, True, cfg)
+    assert bf16_ulp_diff(got, want).max() <= 1
+
+
 # Grids that leave a short last round: its tiles are split into two half-width
 # items (e.g. 12 tiles on 5 CTAs: 10 whole tiles, then 2 tiles as 4 halves).
 TAIL_CASES = [((300, 776, 656), 5), ((300, 776, 656), 9), ((129, 520, 1040), 4), ((260, 1032, 272), 13)]

@@ -76,12 +76,18 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // (cta_group::2), and the narrower 128 x 128 / 256 x 128 tiles, which keep
 // more CTAs busy on small problems but need about twice the operand bytes
 // per multiply-add and measured ~1.7-1.9x slower per operation on B200.
-// Each persistent CTA (pair) does ceil(tiles / units) tiles; a tile costs
-// its multiply-adds times its relative cost, plus a fixed fill / drain
-// overhead of two K blocks.
+// The pair tile is the fastest where K % 128 == 0: it then loads boxes of
+// two K-chunks, which the memory system delivers at ~100 B/clk per SM
+// against the 64 it needs (0.88 of the single-CTA tile's time, measured);
+// otherwise it is on a par with the single-CTA tile.  Each persistent CTA
+// (pair) does ceil(tiles / units) tiles, the last round in half-width items
+// when that leaves at least half the units idle; a tile costs its
+// multiply-adds times its relative cost, plus a fixed fill / drain overhead
+// of two K blocks.
 w8a8_gemm_config select(int64_t M, int64_t N, int64_t K, int sms, bool allow_pair = true) {
   struct Cand { int bm, bn; double rel_cost; int raster; };
-  const Cand cands[4] = {{128, 256, 1.00, 1}, {256, 256, 1.02, 8}, {128, 128, 1.75, 1}, {256, 128, 1.90, 8}};
+  const double pair_cost = K % 128 == 0 ? 0.88 : 1.02;
+  const Cand cands[4] = {{128, 256, 1.00, 1}, {256, 256, pair_cost, 1}, {128, 128, 1.75, 1}, {256, 128, 1.90, 8}};
   double best = 1e300;
   w8a8_gemm_config cfg{};
   const double kblocks = static_cast<double>(ceil_div(K, 128));
@@ -89,9 +95,14 @@ w8a8_gemm_config select(int64_t M, int64_t N, int64_t K, int sms, bool allow_pai
     if (c.bm == 256 && !allow_pair) continue;
     const int units = c.bm == 256 ? sms / 2 : sms;
     const int64_t tiles = ceil_div(M, c.bm) * ceil_div(N, c.bn);
-    const int64_t per_unit = ceil_div(tiles, units);
+    // rounds of tiles per unit; a short last round of 256-column tiles runs
+    // as half-width items (half a round)
+    const int64_t tail = tiles % units;
+    const double per_unit = (c.bn == 256 && tail > 0 && 2 * tail <= units && tiles > units)
+                                ? static_cast<double>(tiles / units) + 0.5
+                                : static_cast<double>(ceil_div(tiles, units));
     const double macs_per_sm = static_cast<double>(c.bm / (c.bm == 256 ? 2 : 1)) * c.bn;
-    const double cost = static_cast<double>(per_unit) * macs_per_sm * (kblocks + 2.0) * c.rel_cost;
+    const double cost = per_unit * macs_per_sm * (kblocks + 2.0) * c.rel_cost;
     if (cost < best * 0.999) {
       best = cost;
       cfg.block_m = c.bm;

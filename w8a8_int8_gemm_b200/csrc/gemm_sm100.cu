@@ -94,11 +94,12 @@ __host__ __device__ constexpr int a_stage_bytes() { return kBlockM * kBlockK; }
 __host__ __device__ constexpr int params_bytes(int bn) { return bn * 6; }
 
 // Dynamic shared memory of one CTA: alignment slack, the operand ring (A:
-// 128 rows, B: block_n rows, or block_n / 2 for a CTA pair), the epilogue's
-// staging blocks and per-tile constants, and the barriers.
-int smem_bytes(bool pair, int bn, int stages) {
+// 128 rows, B: block_n rows, or block_n / 2 for a CTA pair; `chunks` K-chunks
+// of 128 bytes in all), the epilogue's staging blocks and per-tile
+// constants, and the barriers.
+int smem_bytes(bool pair, int bn, int chunks) {
   const int b_rows = pair ? bn / 2 : bn;
-  return 1024 + stages * (a_stage_bytes() + b_rows * kBlockK) + kEpiWarps * kEpiBufBytes + params_bytes(bn) +
+  return 1024 + chunks * (a_stage_bytes() + b_rows * kBlockK) + kEpiWarps * kEpiBufBytes + params_bytes(bn) +
          kBarrierBytes;
 }
 
@@ -177,15 +178,19 @@ __device__ __forceinline__ void dequant_32(const uint32_t (&v)[32], float sa, co
 // A, and the epilogue before reading its scales.  All CTAs are co-resident
 // (cooperative launch), so these waits cannot deadlock; they are bounded
 // all the same.  The last CTA to finish resets the counters to zero.
-template <int BN, GemmOut OUT, bool PAIR, bool FUSE, GemmElem EL>
+template <int BN, GemmOut OUT, bool PAIR, bool FUSE, GemmElem EL, int KCH>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_b_half, const __grid_constant__ CUtensorMap tm_d,
                      const Params p) {
   constexpr int kTileM = PAIR ? 2 * kBlockM : kBlockM;  // rows of the output tile
   constexpr int kBRows = PAIR ? BN / 2 : BN;             // rows of B this CTA loads
-  constexpr uint32_t kA = a_stage_bytes();
-  constexpr uint32_t kB = kBRows * kBlockK;
+  // A ring stage holds KCH K-chunks of 128 bytes of both operands, each
+  // chunk [rows][128 B] (KCH = 2: CTA pairs, loaded as boxes spanning two
+  // chunks through 3-D tensor maps).
+  static_assert(KCH == 1 || (KCH == 2 && PAIR && !FUSE), "double-chunk stages are for CTA pairs");
+  constexpr uint32_t kA = KCH * a_stage_bytes();
+  constexpr uint32_t kB = KCH * kBRows * kBlockK;
   constexpr uint32_t kTxBytes = (PAIR ? 2 : 1) * (kA + kB);
   constexpr uint32_t kTmemCols = 2 * BN;  // two accumulator buffers; 256 or 512 (power of two)
   constexpr bool kE4M3 = EL == GemmElem::kE4M3;
@@ -269,18 +274,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       int mb, nb, hb;
       item_coords(item, p, mb, nb, hb);
       const int a_row = mb * kTileM + static_cast<int>(rank) * kBlockM;
-      const int b_row = nb * BN + (hb < 0 ? static_cast<int>(rank) * kBRows : hb * (BN / 2));
+      // this CTA's rows of B: all BN (single CTA) or its half (pair); a
+      // half-width item covers BN / 2 columns, of which a pair's CTA loads half
+      const int b_row = nb * BN + (hb < 0 ? static_cast<int>(rank) * kBRows
+                                          : hb * (BN / 2) + static_cast<int>(rank) * (kBRows / 2));
       // a half-width item loads half of B's rows, through the tensor map with half-height boxes
       const CUtensorMap* map_b = hb < 0 ? &tm_b : &tm_b_half;
-      const uint32_t tx_bytes = hb < 0 ? kTxBytes : kA + kB / 2;
+      const uint32_t tx_bytes = hb < 0 ? kTxBytes : (PAIR ? 2u : 1u) * (kA + kB / 2);
       for (int kb = 0; kb < p.k_blocks; ++kb) {
         ok = warp_wait(&empty[stage], phase ^ 1u, abort_flag, p.timeout_ns, p.err, kSiteProducerEmpty);
         if (!ok) break;
         if (lane == 0) {
-          if constexpr (PAIR) {
+          if constexpr (PAIR && KCH == 2) {
+            // 3-D maps {128 B, rows, K-chunk}: one box = this CTA's rows x two chunks
             const uint32_t bar = map_to_cta(smem_u32(&full[stage]), 0u);
-            if (leader) mbar_arrive_expect_tx(&full[stage], kTxBytes);
-            tma_load_2d_pair_hint(sB + stage * kB, &tm_b, bar, kb * kBlockK, b_row, keep);
+            if (leader) mbar_arrive_expect_tx(&full[stage], tx_bytes);
+            tma_load_3d_pair_hint(sB + stage * kB, map_b, bar, 0, b_row, 2 * kb, keep);
+            if (fills == 0) pdl_wait_prerequisites();  // A may be written by the kernel before this one
+            tma_load_3d_pair_hint(sA + stage * kA, &tm_a, bar, 0, a_row, 2 * kb, keep);
+          } else if constexpr (PAIR) {
+            const uint32_t bar = map_to_cta(smem_u32(&full[stage]), 0u);
+            if (leader) mbar_arrive_expect_tx(&full[stage], tx_bytes);
+            tma_load_2d_pair_hint(sB + stage * kB, map_b, bar, kb * kBlockK, b_row, keep);
             if (fills == 0) pdl_wait_prerequisites();  // A may be written by the kernel before this one
             tma_load_2d_pair_hint(sA + stage * kA, &tm_a, bar, kb * kBlockK, a_row, keep);
           } else {
@@ -342,6 +357,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int item = unit; ok && item < p.work_items; item += num_units, ++local) {
         const uint32_t idesc = item < p.full_tiles ? kIdesc : kIdescHalf;
+        // bytes between the K-chunks of a stage's B block (half-width items hold half the rows)
+        const uint32_t b_chunk = (item < p.full_tiles ? kBRows : kBRows / 2) * kBlockK;
         const int buf = local & 1;
         const uint32_t tphase = static_cast<uint32_t>(local >> 1) & 1u;
         ok = warp_wait(&tempty[buf], tphase ^ 1u, abort_flag, p.timeout_ns, p.err, kSiteMmaTmemEmpty);
@@ -353,13 +370,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           tc_fence_after_sync();
           if (lane == 0) {
-            const uint64_t a_desc = make_smem_desc_k_sw128(smem_u32(sA + stage * kA));
-            const uint64_t b_desc = make_smem_desc_k_sw128(smem_u32(sB + stage * kB));
 #pragma unroll
-            for (int k = 0; k < kBlockK / kMmaK; ++k) {
-              // Advance the start address by 32 bytes (2 in units of 16 B)
-              // per K=32 slice inside the 128-byte swizzled row.
-              const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+            for (int kk = 0; kk < KCH * (kBlockK / kMmaK); ++kk) {
+              // Chunk c of the stage, then K=32 slice k inside its 128-byte
+              // swizzled rows: the start address advances by 32 bytes (2 in
+              // units of 16 B) per slice.
+              const int c = kk / (kBlockK / kMmaK);
+              const int k = kk % (kBlockK / kMmaK);
+              const uint64_t a_desc =
+                  make_smem_desc_k_sw128(smem_u32(sA + stage * kA + c * a_stage_bytes()));
+              const uint64_t b_desc = make_smem_desc_k_sw128(smem_u32(sB + stage * kB + c * b_chunk));
+              const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
               if constexpr (PAIR && kE4M3) {
                 mma_e4m3_pair(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, acc);
               } else if constexpr (PAIR) {
@@ -657,7 +678,23 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem, const void
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, GemmOut OUT, bool PAIR, bool FUSE, GemmElem EL = GemmElem::kInt8>
+// 3-D view {128 bytes, rows, K / 128} of a K-contiguous byte matrix (K a
+// multiple of 128), boxes of box_rows rows x two K-chunks: one load lands
+// as two [box_rows][128 B] blocks, 128-byte swizzled.
+bool encode_chunks(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr || K % 128 != 0) return false;
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(K / 128)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K), 128};
+  const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows), 2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, GemmOut OUT, bool PAIR, bool FUSE, GemmElem EL = GemmElem::kInt8, int KCH = 1>
 cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t stream) {
   static_assert(!(FUSE && PAIR), "the fused linear layer runs on single CTAs");
   static_assert(!(FUSE && EL == GemmElem::kE4M3), "the fused linear layer is int8 only");
@@ -668,9 +705,15 @@ cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t 
   std::memset(&tm_b, 0, sizeof tm_b);
   std::memset(&tm_b_half, 0, sizeof tm_b_half);
   std::memset(&tm_d, 0, sizeof tm_d);
-  bool ok = encode_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.xq, a.M, a.K, kBlockM, kBlockK) &&
-            encode_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.wq, a.N, a.K, kBRows, kBlockK) &&
-            encode_2d(&tm_b_half, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.wq, a.N, a.K, BN / 2, kBlockK);
+  bool ok;
+  if constexpr (KCH == 2) {
+    ok = encode_chunks(&tm_a, a.xq, a.M, a.K, kBlockM) && encode_chunks(&tm_b, a.wq, a.N, a.K, kBRows) &&
+         encode_chunks(&tm_b_half, a.wq, a.N, a.K, kBRows / 2);
+  } else {
+    ok = encode_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.xq, a.M, a.K, kBlockM, kBlockK) &&
+         encode_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.wq, a.N, a.K, kBRows, kBlockK) &&
+         encode_2d(&tm_b_half, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.wq, a.N, a.K, kBRows / 2, kBlockK);
+  }
   if constexpr (OUT == GemmOut::kBf16Dequant) {
     ok = ok && encode_2d(&tm_d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.out, a.M, a.N, 32, 64);
   } else {
@@ -685,12 +728,12 @@ cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t 
   p.K = static_cast<int>(a.K);
   p.m_tiles = static_cast<int>((a.M + kTileM - 1) / kTileM);
   p.n_tiles = static_cast<int>((a.N + BN - 1) / BN);
-  p.k_blocks = static_cast<int>((a.K + kBlockK - 1) / kBlockK);
+  p.k_blocks = static_cast<int>((a.K + KCH * kBlockK - 1) / (KCH * kBlockK));
   p.num_tiles = p.m_tiles * p.n_tiles;
   p.full_tiles = p.num_tiles;
   p.work_items = p.num_tiles;
   p.raster_group = cfg.raster_group;
-  p.stages = cfg.stages;
+  p.stages = cfg.stages / KCH;  // cfg.stages counts K-chunks of ring depth
   p.scale_a = a.scale_a;
   p.scale_w = a.scale_w;
   p.bias = static_cast<const __nv_bfloat16*>(a.bias);
@@ -704,18 +747,18 @@ cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t 
   cudaError_t e = error_word_address(&p.err);
   if (e != cudaSuccess) return e;
 
-  const int smem = smem_bytes(PAIR, BN, cfg.stages);
-  auto kernel = gemm_w8a8_kernel<BN, OUT, PAIR, FUSE, EL>;
+  const int smem = smem_bytes(PAIR, BN, p.stages * KCH);
+  auto kernel = gemm_w8a8_kernel<BN, OUT, PAIR, FUSE, EL, KCH>;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   // Persistent grid: one CTA (or CTA pair) per tile at most.
   int units = (PAIR ? cfg.grid / 2 : cfg.grid);
   if (units < 1) units = 1;
   if (units > p.num_tiles) units = p.num_tiles;
-  // Last round: if at most half the CTAs would get a tile, give each of the
-  // remaining tiles to two CTAs as half-width items instead.
+  // Last round: if at most half the CTAs (pairs) would get a tile, give each
+  // of the remaining tiles to two CTAs (pairs) as half-width items instead.
   const int tail = p.num_tiles % units;
-  if (!PAIR && BN == 256 && tail > 0 && 2 * tail <= units) {
+  if (BN == 256 && tail > 0 && 2 * tail <= units) {
     p.full_tiles = p.num_tiles - tail;
     p.work_items = p.full_tiles + 2 * tail;
   }
@@ -781,11 +824,22 @@ cudaError_t launch_plain(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t 
   using O = GemmOut;
   const bool bf16 = a.out_kind == O::kBf16Dequant;
   if (cfg.block_m == 256) {
+    // CTA pairs load two K-chunks per box when K allows it and the ring
+    // holds at least two such stages.
+    const bool chunks2 = a.K % 128 == 0 && cfg.stages >= 4;
     if (cfg.block_n == 256) {
+      if (chunks2) {
+        return bf16 ? launch_typed<256, O::kBf16Dequant, true, false, EL, 2>(a, cfg, stream)
+                    : launch_typed<256, O::kAcc32, true, false, EL, 2>(a, cfg, stream);
+      }
       return bf16 ? launch_typed<256, O::kBf16Dequant, true, false, EL>(a, cfg, stream)
                   : launch_typed<256, O::kAcc32, true, false, EL>(a, cfg, stream);
     }
     if (cfg.block_n == 128) {
+      if (chunks2) {
+        return bf16 ? launch_typed<128, O::kBf16Dequant, true, false, EL, 2>(a, cfg, stream)
+                    : launch_typed<128, O::kAcc32, true, false, EL, 2>(a, cfg, stream);
+      }
       return bf16 ? launch_typed<128, O::kBf16Dequant, true, false, EL>(a, cfg, stream)
                   : launch_typed<128, O::kAcc32, true, false, EL>(a, cfg, stream);
     }

@@ -283,6 +283,17 @@ __device__ __forceinline__ void tma_load_2d_pair_hint(void* dst, const void* map
       : "memory");
 }
 
+// 3-D tile load into this CTA's shared memory, completing on an mbarrier of
+// either CTA of the pair, with an L2 eviction-priority policy.
+__device__ __forceinline__ void tma_load_3d_pair_hint(void* dst, const void* map, uint32_t bar_cluster_addr,
+                                                      int32_t x, int32_t y, int32_t z, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar_cluster_addr), "l"(policy)
+      : "memory");
+}
+
 // 2-D tile load into this CTA's shared memory whose byte count completes on
 // an mbarrier of either CTA of the pair (the pair's leader, here).
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const void* map, uint32_t bar_cluster_addr, int32_t x,
