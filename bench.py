@@ -53,6 +53,7 @@ if ROOT not in sys.path:
 import workloads  # noqa: E402
 
 METRIC = "fused W8A8 linear TOPS and % of B200 dense INT8 peak per M×N×K; quantizer GB/s"
+METRIC_BLOCK = "W8A8 DiT-block linear chain TOPS (four linears recorded as one CUDA graph)"
 METRIC_FP8 = "fused W8A8 linear, FP8 (E4M3) variant: TFLOPS and % of B200 dense FP8 peak per M×N×K"
 L2_BYTES = 126 * 1024 * 1024
 NOMINAL_INT8_OVER_BF16 = 2.0     # 4.5 POPS dense int8 / 2.25 PFLOP/s dense bf16 (B200 datasheet)
@@ -607,12 +608,271 @@ def context_baselines(wl, d, sets, sw, bias, dev, args, graph_ms) -> dict:
     return out
 
 
+# ------------------------------------------------------- DiT block chain
+
+
+def oracle_block_sample(blk, rows: int, d: dict, wq: dict) -> float:
+    """Wall time of the oracle running `rows` tokens through every layer of the block."""
+    import oracle
+    sl = slice(0, rows)
+    src = {"x": d["x"][sl], "a": d["a"][sl]}
+    t0 = time.perf_counter()
+    for l in blk.layers:
+        out, _, _, _ = oracle.linear(src[l.source], wq[l.name][0], wq[l.name][1], d["bias_" + l.name])
+        src[l.name] = out
+    return time.perf_counter() - t0
+
+
+def block_oracle_setup(blk, pool_rows: int = 256):
+    import oracle
+    d = blk.inputs(rows=slice(0, pool_rows))
+    wq = {l.name: oracle.quantize_weight(d["w_" + l.name]) for l in blk.layers}
+    return d, wq, oracle.default_threads()
+
+
+def block_cpu_baseline(blk, budget_s: float = 12.0) -> dict:
+    d, wq, cores = block_oracle_setup(blk)
+    t1 = max(oracle_block_sample(blk, 2, d, wq) / 2, 1e-6)
+    rows = int(max(1, min(256, budget_s / t1)))
+    dt = oracle_block_sample(blk, rows, d, wq)
+    ops = blk.ops / blk.M * rows
+    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": cores, "kind": "oracle",
+            "sample": f"{rows} of {blk.M} tokens through all {len(blk.layers)} layers of {blk.name} "
+                      f"(quantize + exact GEMM + epilogue per layer), {dt:.2f} s", "seconds": dt}
+
+
+def run_reference_block(args, blk) -> None:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    d, wq, cores = block_oracle_setup(blk)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    t1 = max(oracle_block_sample(blk, 2, d, wq) / 2, 1e-6)
+    rows = int(max(1, min(256, budget / t1)))
+    for _ in range(args.warmup):
+        oracle_block_sample(blk, rows, d, wq)
+    total = sum(oracle_block_sample(blk, rows, d, wq) for _ in range(args.steps))
+    value = blk.ops / blk.M * rows * args.steps / total / 1e12
+    sample = f"{rows} of {blk.M} tokens through all layers of {blk.name} per step"
+    print(json.dumps({"impl": "reference", "metric": METRIC_BLOCK, "value": value, "unit": "TOPS",
+                      "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                      "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+                      "vs_baseline": None, "dtype": "int64", "data": "synthetic", "config": block_config(blk),
+                      "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores, "kind": "oracle",
+                                       "sample": sample},
+                      "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+                      "gpu_launches": 0}), flush=True)
+
+
+def block_config(blk) -> dict:
+    return {"workload": f"{blk.name}: {blk.note}", "M": blk.M,
+            "layers": [{"name": l.name, "N": l.N, "K": l.K, "input": l.source} for l in blk.layers],
+            "l2": "no rotation needed: one step moves ~0.9 GB, > 7x L2"}
+
+
+def run_block(args, blk) -> None:
+    import w8a8_int8_gemm_b200 as w8
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        _run_block_on(args, blk, w8, rank, world, local, dev, stream)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def _run_block_on(args, blk, w8, rank, world, local, dev, stream) -> None:
+    M = blk.M
+    d = blk.inputs(rows=rank_token_rows(M, rank))
+    host = {k: torch.from_numpy(d[k].view(np.int16)).view(torch.bfloat16) for k in ("x", "a")}
+    src = {k: host[k].to(dev) for k in host}
+    L, wbf16 = {}, {}
+    for l in blk.layers:
+        w32 = torch.from_numpy(d["w_" + l.name]).to(dev)
+        wq, sw = w8.w8a8_quantize_weight(w32)
+        wbf16[l.name] = w32.to(torch.bfloat16)
+        del w32
+        bias = torch.from_numpy(d["bias_" + l.name].view(np.int16)).view(torch.bfloat16).to(dev)
+        L[l.name] = w8.linear_layer(src[l.source], wq, sw, bias)
+        src[l.name] = L[l.name]["out"]
+    chain = w8.w8a8_chain_create([L[l.name] for l in blk.layers])
+    for _ in range(args.warmup):
+        chain.launch(stream)
+    torch.cuda.synchronize(dev)
+    if w8.w8a8_read_device_error() != 0:
+        raise SystemExit("a kernel wait timed out during warm-up")
+
+    def capture(fn, n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+            for i in range(n):
+                fn(i)
+        return g
+
+    # The last R steps of the timed region replay an instrumented graph of
+    # the block with CUDA events around every GEMM launch (the GEMMs then
+    # launch without the programmatic overlap the events would break).
+    R = 3
+    inst_ev = [[(torch.cuda.Event(enable_timing=True, external=True),
+                 torch.cuda.Event(enable_timing=True, external=True)) for _ in blk.layers] for _ in range(R)]
+
+    def step_inst(i):
+        for j, l in enumerate(blk.layers):
+            t = L[l.name]
+            w8.w8a8_quantize_act(t["x"], xq=t["ws_xq"], scale_a=t["ws_scale_a"], stream=stream)
+            inst_ev[i][j][0].record(stream)
+            w8.w8a8_gemm(t["ws_xq"], t["wq"], t["ws_scale_a"], t["scale_w"], t["bias"], out=t["out"], stream=stream)
+            inst_ev[i][j][1].record(stream)
+
+    g_inst = capture(step_inst, R)
+    g_inst.replay()
+    torch.cuda.synchronize(dev)
+    steps = max(args.steps, R + 1)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    start.record(stream)
+    for _ in range(steps - R):
+        chain.launch(stream)
+    g_inst.replay()
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), dev)
+    if w8.w8a8_read_device_error() != 0:
+        raise SystemExit("a kernel wait timed out in the timed region")
+    ms_step = elapsed_ms / steps
+    value = blk.ops * world / (ms_step * 1e-3) / 1e12
+    gemm_ms = {l.name: statistics.fmean(inst_ev[i][j][0].elapsed_time(inst_ev[i][j][1]) for i in range(R))
+               for j, l in enumerate(blk.layers)}
+    gemm_total = sum(gemm_ms.values())
+    kernel_tops = blk.ops / (gemm_total * 1e-3) / 1e12
+
+    peaks = measured_peaks()
+    int8_peak = peaks["bf16_tflops_sustained"] * NOMINAL_INT8_OVER_BF16
+    if rank != 0:
+        chain.close()
+        return
+    G = 10
+
+    def graph_ms(fn, reps=5):
+        g = capture(fn, G)
+        g.replay()
+        a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_ev.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b_ev.record(stream)
+        torch.cuda.synchronize(dev)
+        return a_ev.elapsed_time(b_ev) / (reps * G)
+
+    comps = {"note": "after the timed region, one layer at a time: graphs of back-to-back calls (operands "
+                     "larger than L2 except where noted)"}
+    for l in blk.layers:
+        t = L[l.name]
+        qms = graph_ms(lambda i, t=t: w8.w8a8_quantize_act(t["x"], xq=t["ws_xq"], scale_a=t["ws_scale_a"],
+                                                            stream=stream))
+        lms = graph_ms(lambda i, t=t: w8.w8a8_linear(t["x"], t["wq"], t["scale_w"], t["bias"], out=t["out"],
+                                                      ws_xq=t["ws_xq"], ws_scale_a=t["ws_scale_a"], stream=stream))
+        qbytes = 3 * M * l.K + 4 * M
+        ops = 2.0 * M * l.N * l.K
+        comps[l.name] = {"N": l.N, "K": l.K, "gemm_ms_live": gemm_ms[l.name],
+                         "gemm_tops_live": ops / (gemm_ms[l.name] * 1e-3) / 1e12,
+                         "linear_ms": lms, "quantizer_ms": qms, "quantizer_gbs": qbytes / (qms * 1e-3) / 1e9,
+                         "quantizer_frac_of_measured_hbm": qbytes / (qms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "gemm_config": w8.w8a8_select_config(M, l.N, l.K)}
+    ctx = None
+    if not args.no_context:
+        bsrc = {"x": src["x"], "a": src["a"]}
+        bout = {l.name: torch.empty((M, l.N), dtype=torch.bfloat16, device=dev) for l in blk.layers}
+
+        def bf16_block(i):
+            for l in blk.layers:
+                torch.addmm(L[l.name]["bias"], bsrc[l.source] if l.source in bsrc else bout[l.source],
+                            wbf16[l.name].t(), out=bout[l.name])
+
+        for i in range(2):  # library handles are created outside graph capture
+            bf16_block(i)
+        torch.cuda.synchronize(dev)
+        bms = graph_ms(bf16_block, 3)
+        ctx = {"timing": "CUDA graph of back-to-back blocks", "bf16_matmul_chain": {"ms": bms,
+               "tops": blk.ops / (bms * 1e-3) / 1e12}}
+        del bout
+    e2e = None
+    if args.e2e_steps:
+        pin = {k: host[k].pin_memory() for k in host}
+        outs = [blk.layers[0].name, blk.layers[-1].name]
+        ph = {n: torch.empty((M, L[n]["N"]), dtype=torch.bfloat16).pin_memory() for n in outs}
+
+        def one():
+            for k in pin:
+                src[k].copy_(pin[k], non_blocking=True)
+            chain.launch(stream)
+            for n in outs:
+                ph[n].copy_(L[n]["out"], non_blocking=True)
+
+        for _ in range(3):
+            one()
+        torch.cuda.synchronize(dev)
+        a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_ev.record(stream)
+        for _ in range(args.e2e_steps):
+            one()
+        b_ev.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = a_ev.elapsed_time(b_ev) / args.e2e_steps
+        e2e = {"value": blk.ops / (ems * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": ems,
+               "h2d_bytes_per_step": sum(int(pin[k].numel()) * 2 for k in pin),
+               "d2h_bytes_per_step": sum(int(ph[n].numel()) * 2 for n in outs), "steps": args.e2e_steps,
+               "path": "w8a8_chain_launch with the block inputs copied in and the QKV and MLP-down outputs "
+                       "copied out every step"}
+    cpu = block_cpu_baseline(blk) if (world == 1 and not args.no_cpu_baseline) else None
+    cfg = block_config(blk)
+    cfg["path"] = "w8a8_chain_launch per step: one CUDA graph of 4 x (quantizer + GEMM)"
+    cfg["parallelism"] = f"dp{world} (independent token batches, replicated weights)"
+    cfg["timing"] = (f"{steps} steps between CUDA events; the last {R} replay an instrumented graph with events "
+                     "around each GEMM")
+    result = {
+        "metric": METRIC_BLOCK, "value": value, "unit": "TOPS", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded; stands in for Ideogram 4.0 "
+        "DiT activations and weights, which are not available)", "config": cfg,
+        "roofline": {"bound": "tensor", "achieved": kernel_tops, "peak": int8_peak, "unit": "TOPS",
+                     "frac": kernel_tops / int8_peak, "traffic": None,
+                     "kernel": "gemm_w8a8_kernel over the block's four shapes (sum of their ops / sum of their "
+                               "live launch times)",
+                     "ms_per_launch": gemm_total / len(blk.layers),
+                     "timing": f"CUDA events around each GEMM launch of the last {R} steps of the timed region",
+                     "peak_source": f"{peaks['source']} sustained bf16 {peaks['bf16_tflops_sustained']} TFLOP/s x "
+                                    f"{NOMINAL_INT8_OVER_BF16} (nominal dense int8/bf16 ratio)"},
+        "components": comps, "e2e": e2e, "gpu_launches": 2 * len(blk.layers) * steps, "clocks": clocks,
+        "cpu_baseline": cpu, "context": ctx,
+    }
+    print(json.dumps(result), flush=True)
+    chain.close()
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=12000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default=workloads.HEADLINE,
+                    choices=sorted(workloads.WORKLOADS) + sorted(workloads.BLOCKS),
+                    help="a linear-layer workload, or a DiT block (its linears as one CUDA graph)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--path", default="two-kernel", choices=["fused", "two-kernel"],
@@ -624,6 +884,15 @@ def main(argv=None) -> int:
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.workload in workloads.BLOCKS:
+        blk = workloads.BLOCKS[args.workload]
+        if args.format != "int8" or args.path != "two-kernel":
+            ap.error("the block chain runs the int8 two-kernel layers")
+        if args.impl == "reference":
+            run_reference_block(args, blk)
+        else:
+            run_block(args, blk)
+        return 0
     wl = workloads.WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, wl)

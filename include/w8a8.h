@@ -278,6 +278,53 @@ W8A8_API w8a8_status w8a8_linear_fp8(const void* x, const uint8_t* wq, const flo
                                      int64_t M, int64_t N, int64_t K, w8a8_stream_t stream);
 
 /*
+ * A chain of W8A8 linear layers as one CUDA graph (the paper drops its
+ * kernel into every linear layer of the DiT, abstract; a DiT block runs
+ * four: attention QKV, attention output, MLP up, MLP down).  Each layer is
+ * the w8a8_linear call (activation quantizer, then the GEMM as its
+ * programmatic dependent); w8a8_chain_create records all of them once, in
+ * order, into a CUDA graph, and w8a8_chain_launch replays it with one graph
+ * launch instead of two kernel launches per layer.
+ *
+ * A layer's x may be an earlier layer's out (the same buffer, [M, K] with K
+ * the earlier layer's N): the graph keeps the call order, so the later
+ * quantizer reads the finished output.  All pointers are the caller's
+ * device memory, as for w8a8_linear, and must stay valid, with the same
+ * shapes, for the chain's lifetime: the graph holds the addresses, not
+ * copies.  The chain holds no device memory.  Calls that launch the same
+ * chain (or chains sharing buffers) must not overlap on the GPU.
+ */
+typedef struct {
+    const void* x;            /* bf16 [M, K] input (row stride K) */
+    const int8_t* wq;         /* int8 [N, K] weight codes */
+    const float* scale_w;     /* fp32 [N] */
+    const void* bias;         /* bf16 [N] or NULL */
+    void* out;                /* bf16 [M, N] output (row stride N) */
+    int8_t* ws_xq;            /* int8 [M, K] workspace */
+    float* ws_scale_a;        /* fp32 [M] workspace */
+    int64_t M, N, K;
+} w8a8_linear_desc;
+
+typedef struct w8a8_chain_st* w8a8_chain_t;
+
+/* Validates every layer as w8a8_linear does (errors as for w8a8_linear,
+ * returned before any CUDA call; count must be 1..4096), then records the
+ * chain on the current device.  On success *chain is the new chain; on
+ * failure *chain is NULL and nothing stays allocated. */
+W8A8_API w8a8_status w8a8_chain_create(const w8a8_linear_desc* layers, int32_t count, w8a8_chain_t* chain);
+
+/* Enqueues the whole chain on `stream` (asynchronous, one graph launch).
+ * The current device must be the one the chain was created on. */
+W8A8_API w8a8_status w8a8_chain_launch(w8a8_chain_t chain, w8a8_stream_t stream);
+
+/* Number of layers of the chain (0 for NULL). */
+W8A8_API int32_t w8a8_chain_layers(w8a8_chain_t chain);
+
+/* Frees the chain's graph (NULL is a no-op).  No launch of it may still be
+ * running on the GPU. */
+W8A8_API w8a8_status w8a8_chain_destroy(w8a8_chain_t chain);
+
+/*
  * Every wait inside the library's kernels is bounded in time.  When one
  * runs out the kernel records a nonzero code in a device-side error word,
  * finishes its own in-flight copies, frees its tensor memory and exits, so

@@ -92,6 +92,19 @@ def test_host_validation_without_device(w8):
     assert lib.w8a8_linear_fp8(A, A, A, None, A, A, None, 4, 8, 32, None) == 1    # no ws_scale_a
     cfg = w8.GemmConfig(block_m=256, block_n=256, stages=7, grid=2, raster_group=1)
     assert lib.w8a8_gemm_fp8_f32_ex(A, A, A, 4, 8, 32, ctypes.byref(cfg), None) == 1  # too many stages
+    # chains of linear layers: every layer is validated before any CUDA call
+    h = ctypes.c_void_p(None)
+    assert lib.w8a8_chain_create(None, 1, ctypes.byref(h)) == 1
+    d = (w8.LinearDesc * 2)()
+    d[0] = w8.LinearDesc(A, A, A, None, A, A, A, 4, 8, 32)
+    d[1] = w8.LinearDesc(A, A, A, None, A, A, A, 4, 12, 32)                  # N % 8
+    assert lib.w8a8_chain_create(d, 2, ctypes.byref(h)) == 1 and not h.value
+    d[1] = w8.LinearDesc(A, A, A, None, A, A + 4, A, 4, 8, 32)               # misaligned ws_xq
+    assert lib.w8a8_chain_create(d, 2, ctypes.byref(h)) == 2 and not h.value
+    assert lib.w8a8_chain_create(d, 0, ctypes.byref(h)) == 1
+    assert lib.w8a8_chain_create(d, 1, None) == 1
+    assert lib.w8a8_chain_launch(None, None) == 1
+    assert lib.w8a8_chain_layers(None) == 0 and lib.w8a8_chain_destroy(None) == 0
     # explicit configurations
     cfg = w8.GemmConfig(block_m=128, block_n=200, stages=4, grid=1, raster_group=1)
     assert lib.w8a8_gemm_i32_ex(A, A, A, 4, 8, 32, ctypes.byref(cfg), None) == 1

@@ -45,8 +45,14 @@ def _assert_same(q, s, bits):
     assert bad.size == 0, f"{len(bad)} codes differ, first at {bad[:3].tolist()}"
 
 
+# Every launch path: one-row warps (K <= 4096; 4, 8, 12 and 16 vectors per
+# lane, with M past one wave of resident warps: 4200 x 1024 ... 3000 x 4096);
+# one block per row up to K = 32768 (8, 12 and 16 vectors per thread); the
+# two-pass kernel beyond.
 @pytest.mark.parametrize("M,K", [(1, 16), (7, 48), (9, 272), (63, 1024), (64, 2048), (33, 3072),
-                                 (17, 4096), (5, 4112), (3, 12288), (2, 20000 // 16 * 16)])
+                                 (17, 4096), (5, 4112), (3, 12288), (2, 20000 // 16 * 16), (2369, 1024),
+                                 (4200, 1024), (4500, 2048), (5000, 3072), (3000, 4096), (2, 24576),
+                                 (3, 24592), (2, 40000)])
 def test_act_random_shapes(w8, M, K):
     rng = np.random.default_rng(M * 100003 + K)
     x = rng.standard_normal((M, K)).astype(np.float32) * np.float32(3.0)
@@ -88,7 +94,7 @@ def test_act_workloads_full(w8, name):
 
 
 def test_act_long_k_workload_full(w8):
-    """The 9216 x 12288 input of the MLP down-projection sweep (second-pass path)."""
+    """The 9216 x 12288 input of the MLP down-projection sweep (24 KB rows)."""
     wl = workloads.WORKLOADS["sweep_down"]
     bits = workloads.gen_activations(wl.M, wl.K, wl.seed, wl.outliers)
     q, s = _run_act(w8, bits)
@@ -101,7 +107,7 @@ def test_act_empty(w8):
     assert q.shape == (0, 64) and s.shape == (0,)
 
 
-@pytest.mark.parametrize("N,K", [(128, 256), (136, 48), (12288, 3072), (3072, 12288)])
+@pytest.mark.parametrize("N,K", [(128, 256), (136, 48), (12288, 3072), (3072, 12288), (8, 12304)])
 def test_weight_quant(w8, N, K):
     rng = np.random.default_rng(N + K)
     w = rng.standard_normal((N, K)).astype(np.float32) * np.float32(0.02)

@@ -30,6 +30,8 @@ __all__ = [
     "w8a8_linear_noalloc",
     "w8a8_quantize_act_fp8", "w8a8_quantize_weight_fp8", "w8a8_gemm_fp8", "w8a8_gemm_fp8_ex",
     "w8a8_gemm_fp8_f32", "w8a8_gemm_fp8_f32_ex", "w8a8_linear_fp8",
+    "LinearDesc", "Chain", "linear_layer", "w8a8_chain_create", "w8a8_chain_launch", "w8a8_chain_layers",
+    "w8a8_chain_destroy",
     "w8a8_select_config",
     "w8a8_read_device_error", "w8a8_set_wait_timeout_ns", "w8a8_selftest_wait_timeout",
 ]
@@ -55,6 +57,14 @@ class GemmConfig(ctypes.Structure):
     def as_dict(self) -> dict:
         return {"block_m": self.block_m, "block_n": self.block_n, "stages": self.stages,
                 "grid": self.grid, "raster_group": self.raster_group}
+
+
+class LinearDesc(ctypes.Structure):
+    """w8a8_linear_desc: one layer of a chain (device pointers and sizes)."""
+    _fields_ = [("x", ctypes.c_void_p), ("wq", ctypes.c_void_p), ("scale_w", ctypes.c_void_p),
+                ("bias", ctypes.c_void_p), ("out", ctypes.c_void_p), ("ws_xq", ctypes.c_void_p),
+                ("ws_scale_a", ctypes.c_void_p), ("M", ctypes.c_int64), ("N", ctypes.c_int64),
+                ("K", ctypes.c_int64)]
 
 
 def _load() -> ctypes.CDLL:
@@ -84,6 +94,10 @@ def _load() -> ctypes.CDLL:
         "w8a8_gemm_fp8_f32": ([p, p, p, i64, i64, i64, p], ctypes.c_int),
         "w8a8_gemm_fp8_f32_ex": ([p, p, p, i64, i64, i64, ctypes.POINTER(GemmConfig), p], ctypes.c_int),
         "w8a8_linear_fp8": ([p, p, p, p, p, p, p, i64, i64, i64, p], ctypes.c_int),
+        "w8a8_chain_create": ([ctypes.POINTER(LinearDesc), i32, ctypes.POINTER(p)], ctypes.c_int),
+        "w8a8_chain_launch": ([p, p], ctypes.c_int),
+        "w8a8_chain_layers": ([p], i32),
+        "w8a8_chain_destroy": ([p], ctypes.c_int),
         "w8a8_select_config": ([i64, i64, i64, ctypes.POINTER(GemmConfig)], ctypes.c_int),
         "w8a8_read_device_error": ([ctypes.POINTER(i32), i32], ctypes.c_int),
         "w8a8_set_wait_timeout_ns": ([i64], ctypes.c_int),
@@ -478,6 +492,90 @@ def w8a8_linear_fp8(x, wq, scale_w, bias=None, out=None, ws_xq=None, ws_scale_a=
     _check(_lib.w8a8_linear_fp8(_ptr(x), _ptr(wq), _ptr(scale_w), _ptr(bias), _ptr(out), _ptr(ws_xq),
                                 _ptr(ws_scale_a), M, N, K, _stream(stream, dev)), "w8a8_linear_fp8")
     return out
+
+
+# ------------------------------------------------- chains of linear layers
+
+
+def linear_layer(x, wq, scale_w, bias=None, out=None, ws_xq=None, ws_scale_a=None) -> dict:
+    """One layer of a chain: the tensors of a w8a8_linear call, with the
+    output and workspace allocated here when not given.  x may be an
+    earlier layer's ``out``."""
+    _need(x, "x", torch.bfloat16, 2)
+    M, K = x.shape
+    _need(wq, "wq", torch.int8, 2)
+    N = wq.shape[0]
+    if wq.shape[1] != K:
+        raise ValueError(f"inner dimensions differ: x has K={K}, wq has K={wq.shape[1]}")
+    _need_contig(x, "x", torch.bfloat16, (M, K))
+    _need_contig(wq, "wq", torch.int8, (N, K))
+    _need_contig(scale_w, "scale_w", torch.float32, (N,))
+    if bias is not None:
+        _need_contig(bias, "bias", torch.bfloat16, (N,))
+    dev = x.device
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=dev) if out is None else out
+    ws_xq = torch.empty((M, K), dtype=torch.int8, device=dev) if ws_xq is None else ws_xq
+    ws_scale_a = torch.empty((M,), dtype=torch.float32, device=dev) if ws_scale_a is None else ws_scale_a
+    _need_contig(out, "out", torch.bfloat16, (M, N))
+    _need_contig(ws_xq, "ws_xq", torch.int8, (M, K))
+    _need_contig(ws_scale_a, "ws_scale_a", torch.float32, (M,))
+    return {"x": x, "wq": wq, "scale_w": scale_w, "bias": bias, "out": out, "ws_xq": ws_xq,
+            "ws_scale_a": ws_scale_a, "M": M, "N": N, "K": K}
+
+
+class Chain:
+    """A recorded chain of linear layers (w8a8_chain_t).  Keeps the layers'
+    tensors alive as long as the chain exists; close() frees the graph."""
+
+    def __init__(self, handle: int, layers: list):
+        self._handle = ctypes.c_void_p(handle)
+        self.layers = layers
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        if not self._handle:
+            raise ValueError("the chain has been closed")
+        return self._handle
+
+    def launch(self, stream=None) -> None:
+        w8a8_chain_launch(self, stream)
+
+    def close(self) -> None:
+        if self._handle:
+            st = _lib.w8a8_chain_destroy(self._handle)
+            self._handle = ctypes.c_void_p(None)
+            _check(st, "w8a8_chain_destroy")
+
+    def __del__(self):
+        try:
+            if self._handle:
+                _lib.w8a8_chain_destroy(self._handle)
+        except Exception:  # interpreter shutdown
+            pass
+
+
+def w8a8_chain_create(layers: list) -> Chain:
+    """Record the layers (dicts from linear_layer) as one CUDA graph on the current device."""
+    descs = (LinearDesc * max(1, len(layers)))()
+    for i, l in enumerate(layers):
+        descs[i] = LinearDesc(_ptr(l["x"]), _ptr(l["wq"]), _ptr(l["scale_w"]), _ptr(l.get("bias")), _ptr(l["out"]),
+                              _ptr(l["ws_xq"]), _ptr(l["ws_scale_a"]), l["M"], l["N"], l["K"])
+    h = ctypes.c_void_p(None)
+    _check(_lib.w8a8_chain_create(descs, len(layers), ctypes.byref(h)), "w8a8_chain_create")
+    return Chain(h.value, list(layers))
+
+
+def w8a8_chain_launch(chain: Chain, stream=None) -> None:
+    dev = chain.layers[0]["x"].device if chain.layers else torch.device("cuda")
+    _check(_lib.w8a8_chain_launch(chain.handle, _stream(stream, dev)), "w8a8_chain_launch")
+
+
+def w8a8_chain_layers(chain: Chain) -> int:
+    return int(_lib.w8a8_chain_layers(chain.handle))
+
+
+def w8a8_chain_destroy(chain: Chain) -> None:
+    chain.close()
 
 
 def w8a8_select_config(M: int, N: int, K: int) -> dict:

@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libw8a8.so")
 
-SOURCES = ["api.cu", "quant.cu", "gemm_sm100.cu", "linear_noalloc.cu"]
+SOURCES = ["api.cu", "quant.cu", "gemm_sm100.cu", "linear_noalloc.cu", "chain.cu"]
 HEADERS = ["internal.h", "sm100_ptx.cuh", "quant_row.cuh"]
 
 NVCC_FLAGS = [

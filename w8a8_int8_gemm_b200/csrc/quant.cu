@@ -8,13 +8,17 @@
 //   scale[r] = fl32(max_k |x[r,k]| / 127)
 //   q[r,k]   = clamp(rne(fl32(x[r,k] / scale[r])), -127, 127), 0 if scale[r] == 0
 //
-// Layout: one warp per row.  For rows of up to 32*16 vectors the warp
-// issues every 16-byte load of the row at once and keeps the row in
+// Layout.  Rows of up to 32 * 16 vectors (K <= 4096 bf16): one warp per
+// row, every 16-byte load of the row issued at once and the row kept in
 // registers (blocks of 128 threads, so that all rows of a DiT-sized batch are
-// resident together); longer rows take two passes, the second re-reading the
-// row from L1/L2.  |x| is reduced with a butterfly shuffle; the int8 codes
-// are written packed (8 or 4 bytes per lane per vector).  HBM sees 3 bytes
-// per bf16 element (2 in, 1 out): the kernel is bound by HBM bandwidth.
+// resident together: the bytes in flight, not the instruction count, set
+// the speed of this kernel).  Longer rows, up to 16 vectors per thread of a
+// 256-thread block (K <= 32768 bf16, 16384 fp32): one block per row, the row
+// in the block's registers, |x| reduced across its warps through shared
+// memory, one pass over HBM.  Longer still: a two-pass register kernel that
+// reads the row twice.  |x| is reduced with butterfly shuffles; the codes are
+// written packed (8 or 4 bytes per lane per vector).  HBM sees 3 bytes per
+// bf16 element (2 in, 1 out): the kernels are bound by HBM bandwidth.
 //
 // Exactness.  The code q is decided in binary32 exactly as the definition
 // says.  Instead of one IEEE division per element, the kernel multiplies by
@@ -84,6 +88,52 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict_
   if (lane == 0) scale[row] = s;
 }
 
+// One 256-thread block per row of up to 256 * VPL vectors: the row in the
+// block's registers, |x| reduced over the block through shared memory.
+template <typename T, int VPL, qrow::Code C>
+__global__ void __launch_bounds__(256) quantize_rows_block_kernel(const T* __restrict__ x, int64_t K, int64_t ldx,
+                                                                  int8_t* __restrict__ q, int64_t ldq,
+                                                                  float* __restrict__ scale) {
+  pdl_launch_dependents();
+  constexpr int E = qrow::Vec<T>::kElems;
+  constexpr int kWarps = 8;
+  __shared__ float wmax[kWarps];
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int64_t row = blockIdx.x;
+  const int nvec = static_cast<int>(K / E);
+  const uint4* xr = reinterpret_cast<const uint4*>(x + row * ldx);
+  uint4 c[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int v = tid + 256 * i;
+    c[i] = v < nvec ? __ldg(xr + v) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) amax = fmaxf(amax, qrow::vec_absmax<T>(c[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (lane == 0) wmax[tid >> 5] = amax;
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) amax = fmaxf(amax, wmax[w]);
+  const qrow::RowScale rs = qrow::row_scale<C>(amax);  // every lane holds the row's max
+  int8_t* qr = q + row * ldq;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int v = tid + 256 * i;
+    if (v < nvec) {
+      if (rs.zero) {
+        qrow::store_zero<E>(qr + E * v);
+      } else {
+        qrow::encode_vec<T, C>(c[i], rs, qr + E * v);
+      }
+    }
+  }
+  if (tid == 0) scale[row] = rs.s;
+}
+
 template <typename T, int VPL, qrow::Code C>
 void launch_regs(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq, float* scale,
                  cudaStream_t stream) {
@@ -93,18 +143,40 @@ void launch_regs(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64
       <<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, M, K, ldx, q, ldq, scale);
 }
 
+template <typename T, int VPL, qrow::Code C>
+void launch_block(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq, float* scale,
+                  cudaStream_t stream) {
+  quantize_rows_block_kernel<T, VPL, C><<<static_cast<unsigned>(M), 256, 0, stream>>>(x, K, ldx, q, ldq, scale);
+}
+
 template <typename T, qrow::Code C>
 cudaError_t launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq, float* scale,
                             cudaStream_t stream) {
-  const int64_t per_lane = (K / qrow::Vec<T>::kElems + 31) / 32;
+  const int64_t nvec = K / qrow::Vec<T>::kElems;
+  const int64_t per_lane = (nvec + 31) / 32;
   if (per_lane <= 4) {
     launch_regs<T, 4, C>(x, M, K, ldx, q, ldq, scale, stream);
-  } else if (per_lane <= 8) {
+    return cudaGetLastError();
+  }
+  if (per_lane <= 8) {
     launch_regs<T, 8, C>(x, M, K, ldx, q, ldq, scale, stream);
-  } else if (per_lane <= 12) {
+    return cudaGetLastError();
+  }
+  if (per_lane <= 12) {
     launch_regs<T, 12, C>(x, M, K, ldx, q, ldq, scale, stream);
-  } else if (per_lane <= 16) {
+    return cudaGetLastError();
+  }
+  if (per_lane <= 16) {
     launch_regs<T, 16, C>(x, M, K, ldx, q, ldq, scale, stream);
+    return cudaGetLastError();
+  }
+  const int64_t per_thread = (nvec + 255) / 256;  // one 256-thread block per row
+  if (per_thread <= 8) {
+    launch_block<T, 8, C>(x, M, K, ldx, q, ldq, scale, stream);
+  } else if (per_thread <= 12) {
+    launch_block<T, 12, C>(x, M, K, ldx, q, ldq, scale, stream);
+  } else if (per_thread <= 16) {
+    launch_block<T, 16, C>(x, M, K, ldx, q, ldq, scale, stream);
   } else {
     const int threads = 256;
     const int64_t blocks = (M + (threads / 32) - 1) / (threads / 32);
@@ -134,7 +206,8 @@ cudaError_t launch_quantize_act_e4m3(const void* x, int64_t M, int64_t K, int64_
 
 cudaError_t launch_quantize_weight_e4m3(const float* w, int64_t N, int64_t K, int64_t ldw, uint8_t* q, int64_t ldq,
                                         float* scale, cudaStream_t stream) {
-  return launch_quantize<float, qrow::Code::kE4M3>(w, N, K, ldw, reinterpret_cast<int8_t*>(q), ldq, scale, stream);
+  return launch_quantize<float, qrow::Code::kE4M3>(w, N, K, ldw, reinterpret_cast<int8_t*>(q), ldq, scale, 
+                                                   stream);
 }
 
 }  // namespace w8a8

@@ -78,6 +78,57 @@ WORKLOADS: dict[str, Workload] = {w.name: w for w in [
 HEADLINE = "mlp_up_1024"
 
 
+@dataclass(frozen=True)
+class BlockLayer:
+    name: str
+    N: int
+    K: int
+    source: str           # "x" / "a": a block input; otherwise the name of the layer whose output feeds it
+
+
+@dataclass(frozen=True)
+class Block:
+    """The linear layers of one DiT block over M tokens, in execution order.
+    Inputs "x" (the block input) and "a" (the attention result feeding the
+    attention output projection) are seeded bf16 N(0, 1); the norm,
+    attention and GELU between the linears are not part of the method, so
+    MLP up reads the attention output projection's result directly and MLP
+    down reads MLP up's."""
+    name: str
+    index: int
+    M: int
+    layers: tuple
+    note: str = ""
+
+    @property
+    def seed(self) -> int:
+        return SEED_BASE + self.index
+
+    @property
+    def ops(self) -> int:
+        return sum(2 * self.M * l.N * l.K for l in self.layers)
+
+    def inputs(self, rows: slice | None = None) -> dict:
+        """Seeded host inputs: x, a (bf16 bits, rows of the token stream),
+        per layer w (fp32) and bias (bf16 bits)."""
+        r0 = 0 if rows is None else rows.start
+        m = self.M if rows is None else rows.stop - rows.start
+        d = {"x": gen_activations(m, self.layers[0].K, self.seed, row_offset=r0),
+             "a": gen_activations(m, 3072, self.seed + 100, row_offset=r0)}
+        for i, l in enumerate(self.layers):
+            d["w_" + l.name] = gen_weight(l.N, l.K, self.seed + 10 + i)
+            d["bias_" + l.name] = gen_bias(l.N, self.seed + 20 + i)
+        return d
+
+
+BLOCKS: dict[str, Block] = {b.name: b for b in [
+    Block("dit_block_1024", 6, 9216,
+          (BlockLayer("qkv", 9216, 3072, "x"), BlockLayer("attn_out", 3072, 3072, "a"),
+           BlockLayer("mlp_up", 12288, 3072, "attn_out"), BlockLayer("mlp_down", 3072, 12288, "mlp_up")),
+          note="the four linears of one DiT block, batch 2 at 1024px + 512 text tokens (M = 9216)"),
+]}
+
+
 def _to_bf16_bits(a: np.ndarray) -> np.ndarray:
     """float32 array -> bf16 bit patterns (uint16), by torch's CPU rounding."""
     t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
