@@ -513,41 +513,71 @@ def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
 
 
 def run_e2e(w8, wl, x_host, wq, sw, bias, dev, stream, args) -> dict:
-    """The public API with host buffers: pinned host X -> device, w8a8_linear,
-    result -> pinned host, every step, timed on the device."""
+    """The public API with host buffers, every step: its input X copied in
+    from pinned host memory, the linear layer, its output copied back to
+    pinned host memory; timed on the device from the first copy in to the
+    last copy out.  Steps are pipelined as a serving loop would run them:
+    three streams (copy in, compute, copy out) and two buffer sets, so step
+    i+1's copy in and step i-1's copy out overlap step i's compute (PCIe is
+    full duplex); event dependencies keep every buffer's reuse safe."""
     M, N, K = wl.M, wl.N, wl.K
-    xh = x_host.pin_memory()
-    oh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-    xd = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
-    od = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     fp8 = args.format == "fp8"
+    linear = w8.w8a8_linear_fp8 if fp8 else w8.w8a8_linear
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    B = 2
+    xh = [x_host.pin_memory() for _ in range(B)]
+    oh = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(B)]
+    xd = [torch.empty((M, K), dtype=torch.bfloat16, device=dev) for _ in range(B)]
+    od = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(B)]
     xq = torch.empty((M, K), dtype=torch.uint8 if fp8 else torch.int8, device=dev)
     sa = torch.empty((M,), dtype=torch.float32, device=dev)
     sync = torch.zeros((w8.w8a8_linear_sync_words(M),), dtype=torch.int32, device=dev)
-    linear = w8.w8a8_linear_fp8 if fp8 else w8.w8a8_linear
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    copied_in = [ev() for _ in range(B)]
+    computed = [ev() for _ in range(B)]
+    copied_out = [ev() for _ in range(B)]
+    used = [False] * B
 
-    def one():
-        xd.copy_(xh, non_blocking=True)
+    def one(i):
+        b = i % B
+        if used[b]:
+            s_in.wait_event(computed[b])        # xd[b] is free once step i-B's layer has read it
+        with torch.cuda.stream(s_in):
+            xd[b].copy_(xh[b], non_blocking=True)
+        copied_in[b].record(s_in)
+        stream.wait_event(copied_in[b])
+        if used[b]:
+            stream.wait_event(copied_out[b])    # od[b] is free once step i-B's result is copied out
         if args.path == "fused":
-            w8.w8a8_linear_fused(xd, wq, sw, bias, out=od, ws_xq=xq, ws_scale_a=sa, ws_sync=sync, stream=stream)
+            w8.w8a8_linear_fused(xd[b], wq, sw, bias, out=od[b], ws_xq=xq, ws_scale_a=sa, ws_sync=sync,
+                                 stream=stream)
         else:
-            linear(xd, wq, sw, bias, out=od, ws_xq=xq, ws_scale_a=sa, stream=stream)
-        oh.copy_(od, non_blocking=True)
+            linear(xd[b], wq, sw, bias, out=od[b], ws_xq=xq, ws_scale_a=sa, stream=stream)
+        computed[b].record(stream)
+        s_out.wait_event(computed[b])
+        with torch.cuda.stream(s_out):
+            oh[b].copy_(od[b], non_blocking=True)
+        copied_out[b].record(s_out)
+        used[b] = True
 
-    for _ in range(3):
-        one()
+    for i in range(3):
+        one(i)
     torch.cuda.synchronize(dev)
     steps = args.e2e_steps
     a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        one()
-    b.record(stream)
+    b_ev = torch.cuda.Event(enable_timing=True)
+    a.record(s_in)
+    stream.wait_event(a)
+    s_out.wait_event(a)
+    for i in range(steps):
+        one(i)
+    s_in.wait_event(copied_out[(steps - 1) % B])
+    b_ev.record(s_in)
     torch.cuda.synchronize(dev)
-    ms = a.elapsed_time(b) / steps
+    ms = a.elapsed_time(b_ev) / steps
     return {"value": 2.0 * M * N * K / (ms * 1e-3) / 1e12, "unit": "TFLOPS" if fp8 else "TOPS", "ms_per_step": ms,
-            "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "steps": steps}
+            "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "steps": steps,
+            "pipeline": "copy in / compute / copy out on three streams, two buffer sets"}
 
 
 def context_baselines(wl, d, sets, sw, bias, dev, args, graph_ms) -> dict:
@@ -662,6 +692,82 @@ def run_reference_block(args, blk) -> None:
                                        "sample": sample},
                       "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
                       "gpu_launches": 0}), flush=True)
+
+
+def block_e2e(args, blk, w8, L, host, dev, stream) -> dict:
+    """The block through the chain API with host buffers, every step: the
+    two block inputs copied in from pinned host memory, one chain launch,
+    the QKV and MLP-down outputs copied back.  Pipelined like run_e2e: three
+    streams, two chains recorded over two sets of input/output buffers (the
+    weights, workspaces and the intermediate activations are shared; the
+    compute stream runs the chains one after the other)."""
+    first, last = blk.layers[0].name, blk.layers[-1].name
+    B = 2
+    ins, outs, chains = [], [], []
+    for b in range(B):
+        src = {k: torch.empty_like(L[blk.layers[0].name]["x"]) if k == "x" else torch.empty(
+            (blk.M, 3072), dtype=torch.bfloat16, device=dev) for k in ("x", "a")}
+        layers = []
+        for l in blk.layers:
+            t = L[l.name]
+            out = torch.empty_like(t["out"]) if l.name in (first, last) else t["out"]
+            x = src[l.source] if l.source in src else layers[[m.name for m in blk.layers].index(l.source)]["out"]
+            layers.append(w8.linear_layer(x, t["wq"], t["scale_w"], t["bias"], out=out, ws_xq=t["ws_xq"],
+                                          ws_scale_a=t["ws_scale_a"]))
+        ins.append(src)
+        outs.append({first: layers[0]["out"], last: layers[-1]["out"]})
+        chains.append(w8.w8a8_chain_create(layers))
+    pin = [{k: host[k].pin_memory() for k in host} for _ in range(B)]
+    ph = [{n: torch.empty(tuple(outs[0][n].shape), dtype=torch.bfloat16).pin_memory() for n in (first, last)}
+          for _ in range(B)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    copied_in = [torch.cuda.Event() for _ in range(B)]
+    computed = [torch.cuda.Event() for _ in range(B)]
+    copied_out = [torch.cuda.Event() for _ in range(B)]
+    used = [False] * B
+
+    def one(i):
+        b = i % B
+        if used[b]:
+            s_in.wait_event(computed[b])
+        with torch.cuda.stream(s_in):
+            for k in pin[b]:
+                ins[b][k].copy_(pin[b][k], non_blocking=True)
+        copied_in[b].record(s_in)
+        stream.wait_event(copied_in[b])
+        if used[b]:
+            stream.wait_event(copied_out[b])
+        chains[b].launch(stream)
+        computed[b].record(stream)
+        s_out.wait_event(computed[b])
+        with torch.cuda.stream(s_out):
+            for n in ph[b]:
+                ph[b][n].copy_(outs[b][n], non_blocking=True)
+        copied_out[b].record(s_out)
+        used[b] = True
+
+    for i in range(3):
+        one(i)
+    torch.cuda.synchronize(dev)
+    steps = args.e2e_steps
+    a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a_ev.record(s_in)
+    stream.wait_event(a_ev)
+    s_out.wait_event(a_ev)
+    for i in range(steps):
+        one(i)
+    s_in.wait_event(copied_out[(steps - 1) % B])
+    b_ev.record(s_in)
+    torch.cuda.synchronize(dev)
+    for c in chains:
+        c.close()
+    ems = a_ev.elapsed_time(b_ev) / steps
+    return {"value": blk.ops / (ems * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": ems,
+            "h2d_bytes_per_step": sum(int(pin[0][k].numel()) * 2 for k in pin[0]),
+            "d2h_bytes_per_step": sum(int(ph[0][n].numel()) * 2 for n in ph[0]), "steps": steps,
+            "path": "w8a8_chain_launch with the block inputs copied in and the QKV and MLP-down outputs copied "
+                    "out every step",
+            "pipeline": "copy in / compute / copy out on three streams, two chains over two buffer sets"}
 
 
 def block_config(blk) -> dict:
@@ -813,32 +919,7 @@ def _run_block_on(args, blk, w8, rank, world, local, dev, stream) -> None:
         del bout
     e2e = None
     if args.e2e_steps:
-        pin = {k: host[k].pin_memory() for k in host}
-        outs = [blk.layers[0].name, blk.layers[-1].name]
-        ph = {n: torch.empty((M, L[n]["N"]), dtype=torch.bfloat16).pin_memory() for n in outs}
-
-        def one():
-            for k in pin:
-                src[k].copy_(pin[k], non_blocking=True)
-            chain.launch(stream)
-            for n in outs:
-                ph[n].copy_(L[n]["out"], non_blocking=True)
-
-        for _ in range(3):
-            one()
-        torch.cuda.synchronize(dev)
-        a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a_ev.record(stream)
-        for _ in range(args.e2e_steps):
-            one()
-        b_ev.record(stream)
-        torch.cuda.synchronize(dev)
-        ems = a_ev.elapsed_time(b_ev) / args.e2e_steps
-        e2e = {"value": blk.ops / (ems * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": ems,
-               "h2d_bytes_per_step": sum(int(pin[k].numel()) * 2 for k in pin),
-               "d2h_bytes_per_step": sum(int(ph[n].numel()) * 2 for n in outs), "steps": args.e2e_steps,
-               "path": "w8a8_chain_launch with the block inputs copied in and the QKV and MLP-down outputs "
-                       "copied out every step"}
+        e2e = block_e2e(args, blk, w8, L, host, dev, stream)
     cpu = block_cpu_baseline(blk) if (world == 1 and not args.no_cpu_baseline) else None
     cfg = block_config(blk)
     cfg["path"] = "w8a8_chain_launch per step: one CUDA graph of 4 x (quantizer + GEMM)"
