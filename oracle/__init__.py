@@ -81,9 +81,19 @@ class Oracle:
         lib.oracle_quantize_rows_f32_fp8.argtypes = [p, i64, i64, i64, p, i64, p]
         lib.oracle_gemm_fp8_f64.argtypes = [p, p, i64, i64, i64, p]
         lib.oracle_epilogue_fp8.argtypes = [p, p, p, p, i64, i64, p]
+        lib.oracle_expf.argtypes = [ctypes.c_float]
+        lib.oracle_expf.restype = ctypes.c_float
+        lib.oracle_gelu_f32.argtypes = [ctypes.c_float]
+        lib.oracle_gelu_f32.restype = ctypes.c_float
+        lib.oracle_expf_array.argtypes = [p, i64, p]
+        lib.oracle_expf_array.restype = None
+        lib.oracle_gelu_f32_array.argtypes = [p, i64, p]
+        lib.oracle_gelu_f32_array.restype = None
+        lib.oracle_gelu_rows.argtypes = [p, i64, i64, i64, p, i64]
         for fn in ("oracle_quantize_rows_bf16", "oracle_quantize_rows_f32", "oracle_gemm_i64",
                    "oracle_epilogue", "oracle_epilogue_f64", "oracle_linear", "oracle_quantize_rows_bf16_fp8",
-                   "oracle_quantize_rows_f32_fp8", "oracle_gemm_fp8_f64", "oracle_epilogue_fp8"):
+                   "oracle_quantize_rows_f32_fp8", "oracle_gemm_fp8_f64", "oracle_epilogue_fp8",
+                   "oracle_gelu_rows"):
             getattr(lib, fn).restype = ctypes.c_int
         self.lib = lib
         self.path = libpath
@@ -282,6 +292,35 @@ class Oracle:
         return out
 
 
+    # --------------------------------------- GELU (producer of X), fused quantizer
+
+    def expf(self, x) -> np.ndarray:
+        """The oracle's own binary32 exp, element-wise."""
+        a = _c(x, np.float32)
+        y = np.empty_like(a)
+        self.lib.oracle_expf_array(_ptr(a), a.size, _ptr(y))
+        return y
+
+    def gelu_f32(self, x) -> np.ndarray:
+        """GELU (tanh form) in binary32, element-wise, before any bf16 rounding."""
+        a = _c(x, np.float32)
+        y = np.empty_like(a)
+        self.lib.oracle_gelu_f32_array(_ptr(a), a.size, _ptr(y))
+        return y
+
+    def gelu(self, h_bits) -> np.ndarray:
+        """bf16 bits [M, K] -> bf16 bits of bf16_rne(GELU(h))."""
+        h = _c(h_bits, np.uint16)
+        M, K = h.shape
+        g = np.empty((M, K), np.uint16)
+        self._check(self.lib.oracle_gelu_rows(_ptr(h), M, K, K, _ptr(g), K), "gelu_rows")
+        return g
+
+    def gelu_quantize_act(self, h_bits):
+        """The per-token quantizer applied to bf16_rne(GELU(h)): (codes, scales)."""
+        return self.quantize_act(self.gelu(h_bits))
+
+
 _default: Oracle | None = None
 
 
@@ -347,3 +386,19 @@ def gemm_fp8(aq, bq):
 
 def epilogue_fp8(acc, scale_a, scale_w, bias_bits=None):
     return get().epilogue_fp8(acc, scale_a, scale_w, bias_bits)
+
+
+def expf(x):
+    return get().expf(x)
+
+
+def gelu_f32(x):
+    return get().gelu_f32(x)
+
+
+def gelu(h_bits):
+    return get().gelu(h_bits)
+
+
+def gelu_quantize_act(h_bits):
+    return get().gelu_quantize_act(h_bits)

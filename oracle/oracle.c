@@ -38,6 +38,13 @@
  *   acc[m,n]  = sum_k e4m3(q_x[m,k]) * e4m3(q_w[n,k])   (exact, here in binary64)
  *   out[m,n]  = bf16_rne( fl32( fl32( fl32(acc)*s_a[m] ) * s_w[n] ) + bias[n] )
  *
+ * GELU before a linear layer (the producer of its input, fused with the
+ * per-token quantizer on the GPU): the tanh form h / (1 + exp(-2u)),
+ * u = sqrt(2/pi) (h + 0.044715 h^3), with this file's own exp (Cody-Waite
+ * reduction and a degree-7 Taylor polynomial), rounded to bf16:
+ *
+ *   g[r,k]    = bf16_rne( gelu(h[r,k]) ),  then the quantizer above on g
+ *
  * Parity pins (what this file is checked against, other than itself):
  * brute force and closed forms in the CPU test suite -- numpy float32
  * division and rint for the quantizer, numpy int64 matmul and exact
@@ -185,6 +192,73 @@ int oracle_epilogue_fp8(const double* acc, const float* scale_a, const float* sc
             float bn = bias ? oracle_bf16_to_f32(bias[n]) : 0.0f;
             out[m * N + n] = oracle_f32_to_bf16_rne(d + bn);
         }
+    return 0;
+}
+
+/* ------------------------------------------------- GELU, the producer of X */
+
+/* exp(x) in binary32, this library's own: Cody-Waite reduction
+ * x = k ln2 + r with ln2 split as LN2_HI (low bits zero, so k * LN2_HI is
+ * exact for |k| < 2^9) + LN2_LO, k = rint(x * log2 e); the degree-7 Taylor
+ * polynomial of exp(r) (|r| <= ln2 / 2 + rounding) by Horner's rule with
+ * fused multiply-adds; then one product with 2^k built from its bits.
+ * Arguments above 88 give +inf, below -30 give 0 (1 + exp(x) is 1 in
+ * binary32 there).  Every step one correctly rounded binary32 operation, in
+ * this order, so the GPU reproduces it bit for bit. */
+static const float LOG2E = 1.44269502162933349609375f;    /* fl32(log2 e) */
+static const float LN2_HI = 0.693145751953125f;           /* 0x3F317200 */
+static const float LN2_LO = 1.428606765330187045037746429443359375e-6f;  /* fl32(ln2 - LN2_HI) */
+
+float oracle_expf(float x) {
+    if (x > 88.0f) return INFINITY;
+    if (x < -30.0f) return 0.0f;
+    float k = rintf(x * LOG2E);
+    float r = fmaf(-k, LN2_HI, x);
+    r = fmaf(-k, LN2_LO, r);
+    float p = 1.0f / 5040.0f;
+    p = fmaf(p, r, 1.0f / 720.0f);
+    p = fmaf(p, r, 1.0f / 120.0f);
+    p = fmaf(p, r, 1.0f / 24.0f);
+    p = fmaf(p, r, 1.0f / 6.0f);
+    p = fmaf(p, r, 0.5f);
+    p = fmaf(p, r, 1.0f);
+    p = fmaf(p, r, 1.0f);
+    uint32_t bits = (uint32_t)((int32_t)k + 127) << 23;   /* 2^k, k in [-44, 127] */
+    float scale;
+    memcpy(&scale, &bits, sizeof scale);
+    return p * scale;
+}
+
+/* GELU, tanh form (Hendrycks & Gimpel, "Gaussian Error Linear Units"):
+ * 0.5 h (1 + tanh(u)) = h / (1 + exp(-2u)), u = sqrt(2/pi) (h + 0.044715 h^3),
+ * each operation rounded to binary32 in the order written. */
+static const float GELU_C0 = 0.79788458347320556640625f;  /* fl32(sqrt(2 / pi)) */
+static const float GELU_C1 = 0.044715f;
+
+float oracle_gelu_f32(float h) {
+    float h3 = (h * h) * h;
+    float inner = h + GELU_C1 * h3;
+    float u = GELU_C0 * inner;
+    float e = oracle_expf(-2.0f * u);
+    return h / (1.0f + e);
+}
+
+/* Element-wise over arrays (for the checks of these two functions). */
+void oracle_expf_array(const float* x, int64_t n, float* y) {
+    for (int64_t i = 0; i < n; ++i) y[i] = oracle_expf(x[i]);
+}
+
+void oracle_gelu_f32_array(const float* x, int64_t n, float* y) {
+    for (int64_t i = 0; i < n; ++i) y[i] = oracle_gelu_f32(x[i]);
+}
+
+/* g = bf16_rne(GELU(h)) for bf16 rows h [M, K] (row stride ldh) into g
+ * (row stride ldg): what a GELU kernel writes for the next linear layer. */
+int oracle_gelu_rows(const uint16_t* h, int64_t M, int64_t K, int64_t ldh, uint16_t* g, int64_t ldg) {
+    if (M < 0 || K < 0 || ldh < K || ldg < K) return 1;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < K; ++k)
+            g[m * ldg + k] = oracle_f32_to_bf16_rne(oracle_gelu_f32(oracle_bf16_to_f32(h[m * ldh + k])));
     return 0;
 }
 

@@ -15,6 +15,7 @@ per-token x per-channel dequantization plus bias in the epilogue, bf16 out.
 """
 from __future__ import annotations
 
+import math
 import os
 from fractions import Fraction
 
@@ -476,3 +477,88 @@ def check_fp8_epilogue(orc) -> None:
 
 ALL_CHECKS += [check_e4m3_decode, check_e4m3_encode, check_fp8_quant_golden, check_fp8_quant_vs_library,
                check_fp8_quant_invariants, check_fp8_gemm, check_fp8_epilogue]
+
+
+# ------------------------------------------------- GELU before a linear layer
+
+
+def check_own_expf(orc) -> None:
+    """The oracle's binary32 exp against numpy's float64 exp: within 1 ulp on
+    [-30, 88]; exact at 0; +inf above 88; 0 below -30."""
+    x = np.concatenate([np.linspace(-30, 88, 200001), np.log(2.0) * np.arange(-43, 127)]).astype(np.float32)
+    y = orc.expf(x).astype(np.float64)
+    t = np.exp(x.astype(np.float64))
+    ulp = np.spacing(t.astype(np.float32)).astype(np.float64)
+    assert (np.abs(y - t) <= ulp).all(), float((np.abs(y - t) / ulp).max())
+    edge = orc.expf(np.array([0.0, 88.5, 1e30, -30.5, -1e30], np.float32))
+    assert edge[0] == 1.0 and np.isinf(edge[1]) and np.isinf(edge[2]) and edge[3] == 0.0 and edge[4] == 0.0
+
+
+def _gelu_f64(h: np.ndarray) -> np.ndarray:
+    hd = h.astype(np.float64)
+    u = math.sqrt(2 / math.pi) * (hd + 0.044715 * hd ** 3)
+    with np.errstate(over="ignore"):
+        return hd / (1.0 + np.exp(-2.0 * u)), u
+
+
+def check_gelu_f32(orc) -> None:
+    """GELU (tanh form) against the float64 formula h / (1 + exp(-2u)) within
+    the binary32 error budget: u carries <= 7 roundings' relative error, which
+    exp turns into 14|u| ulp of relative error, plus 8 ulp for the rest; below
+    2^-122 in magnitude the cutoff of exp at 88 may give 0.  Closed forms:
+    gelu(0) = 0, gelu(h) = h exactly for h >= 10 (exp(-2u) < 2^-25), gelu(h)
+    = -0 for h <= -13 (exp argument above 88)."""
+    h = np.concatenate([np.linspace(-20, 20, 400001), np.linspace(-1e-3, 1e-3, 20001),
+                        np.geomspace(1e-30, 1e4, 20000), -np.geomspace(1e-30, 1e4, 20000)]).astype(np.float32)
+    g = orc.gelu_f32(h).astype(np.float64)
+    gt, u = _gelu_f64(h)
+    bound = (14 * np.abs(u) + 8) * 2.0 ** -24 * np.abs(gt) + 2.0 ** -122
+    assert (np.abs(g - gt) <= bound).all(), float((np.abs(g - gt) / bound).max())
+    big = np.linspace(10, 3e38, 1001).astype(np.float32)
+    assert np.array_equal(orc.gelu_f32(big), big)
+    neg = orc.gelu_f32(-np.linspace(13, 3e38, 1001).astype(np.float32))
+    assert (neg == 0).all() and np.signbit(neg).all()
+    assert orc.gelu_f32(np.array([0.0], np.float32))[0] == 0.0
+
+
+def check_gelu_bf16_vs_torch(orc) -> None:
+    """bf16_rne(GELU(h)) against torch's tanh-approximate GELU in float32
+    rounded to bf16 (an independent implementation with its own tanh): within
+    one bf16 ulp, and equal almost everywhere, for h >= -3.  Below that,
+    torch's 0.5 h (1 + tanh(u)) cancels (tanh(u) -> -1) and loses the value
+    the float64 check above holds this function to."""
+    rng = np.random.default_rng(31)
+    x = np.concatenate([rng.standard_normal(200000) * 3, np.linspace(-3, 12, 50001)]).astype(np.float32)
+    x = x[x >= -3]
+    bits = to_bits(x)
+    mine = orc.gelu(bits[None, :])[0]
+    ref = torch.nn.functional.gelu(torch.from_numpy(bits_to_float(bits)), approximate="tanh")
+    ref_bits = ref.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+    def order(b):
+        b = b.astype(np.int32)
+        return np.where(b >= 0x8000, -(b & 0x7FFF), b)
+
+    d = np.abs(order(mine) - order(ref_bits))
+    assert d.max() <= 1, int(d.max())
+    assert (d == 0).mean() > 0.995
+
+
+def check_gelu_quantize(orc) -> None:
+    """The fused producer step is the quantizer applied to the bf16 GELU
+    output: the quantizer's own invariants hold on it (absmax of GELU(h) maps
+    to +-127; rows of large negative h give GELU -0 and an all-zero row)."""
+    rng = np.random.default_rng(32)
+    h = to_bits((rng.standard_normal((16, 256)) * 4).astype(np.float32))
+    h[3, :] = to_bits(np.full(256, -20.0, np.float32))
+    q, s = orc.gelu_quantize_act(h)
+    g = bits_to_float(orc.gelu(h))
+    assert s[3] == 0.0 and (q[3] == 0).all()
+    for r in range(16):
+        if s[r] > 0:
+            assert np.abs(q[r]).max() == 127
+            k = np.abs(g[r]).argmax()
+            assert abs(int(q[r, k])) == 127
+
+
+ALL_CHECKS += [check_own_expf, check_gelu_f32, check_gelu_bf16_vs_torch, check_gelu_quantize]

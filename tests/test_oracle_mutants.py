@@ -51,6 +51,16 @@ MUTANTS = [
      "s += lut[a[m * K + k]] * lut[b[n * K + (K - 1 - k)]];"),
     ("e4m3 epilogue scale_w twice", "d *= scale_a[m];", "d *= scale_w[n];"),
     ("e4m3 epilogue dropped bias", "oracle_f32_to_bf16_rne(d + bn);", "oracle_f32_to_bf16_rne(d);"),
+    # GELU before a linear layer, and its exp
+    ("gelu cubic coefficient 0.04471", "static const float GELU_C1 = 0.044715f;",
+     "static const float GELU_C1 = 0.04471f;"),
+    ("gelu without the cubic term", "float inner = h + GELU_C1 * h3;", "float inner = h;"),
+    ("gelu wrong sign in exp", "float e = oracle_expf(-2.0f * u);", "float e = oracle_expf(2.0f * u);"),
+    ("gelu 1 - e", "return h / (1.0f + e);", "return h / (1.0f - e);"),
+    ("exp without the low part of ln2", "r = fmaf(-k, LN2_LO, r);", ""),
+    ("exp Taylor term r^7 dropped", "float p = 1.0f / 5040.0f;", "float p = 0.0f;"),
+    ("exp scale off by one", "uint32_t bits = (uint32_t)((int32_t)k + 127) << 23;",
+     "uint32_t bits = (uint32_t)((int32_t)k + 128) << 23;"),
 ]
 
 
