@@ -648,7 +648,8 @@ def oracle_block_sample(blk, rows: int, d: dict, wq: dict) -> float:
     src = {"x": d["x"][sl], "a": d["a"][sl]}
     t0 = time.perf_counter()
     for l in blk.layers:
-        out, _, _, _ = oracle.linear(src[l.source], wq[l.name][0], wq[l.name][1], d["bias_" + l.name])
+        x = oracle.gelu(src[l.source]) if l.act == "gelu" else src[l.source]
+        out, _, _, _ = oracle.linear(x, wq[l.name][0], wq[l.name][1], d["bias_" + l.name])
         src[l.name] = out
     return time.perf_counter() - t0
 
@@ -713,7 +714,7 @@ def block_e2e(args, blk, w8, L, host, dev, stream) -> dict:
             out = torch.empty_like(t["out"]) if l.name in (first, last) else t["out"]
             x = src[l.source] if l.source in src else layers[[m.name for m in blk.layers].index(l.source)]["out"]
             layers.append(w8.linear_layer(x, t["wq"], t["scale_w"], t["bias"], out=out, ws_xq=t["ws_xq"],
-                                          ws_scale_a=t["ws_scale_a"]))
+                                          ws_scale_a=t["ws_scale_a"], input_act=t["input_act"]))
         ins.append(src)
         outs.append({first: layers[0]["out"], last: layers[-1]["out"]})
         chains.append(w8.w8a8_chain_create(layers))
@@ -772,7 +773,8 @@ def block_e2e(args, blk, w8, L, host, dev, stream) -> dict:
 
 def block_config(blk) -> dict:
     return {"workload": f"{blk.name}: {blk.note}", "M": blk.M,
-            "layers": [{"name": l.name, "N": l.N, "K": l.K, "input": l.source} for l in blk.layers],
+            "layers": [{"name": l.name, "N": l.N, "K": l.K, "input": l.source + (" (GELU)" if l.act else "")}
+                       for l in blk.layers],
             "l2": "no rotation needed: one step moves ~0.9 GB, > 7x L2"}
 
 
@@ -806,7 +808,8 @@ def _run_block_on(args, blk, w8, rank, world, local, dev, stream) -> None:
         wbf16[l.name] = w32.to(torch.bfloat16)
         del w32
         bias = torch.from_numpy(d["bias_" + l.name].view(np.int16)).view(torch.bfloat16).to(dev)
-        L[l.name] = w8.linear_layer(src[l.source], wq, sw, bias)
+        L[l.name] = w8.linear_layer(src[l.source], wq, sw, bias,
+                                    input_act=w8.ACT_GELU if l.act == "gelu" else w8.ACT_NONE)
         src[l.name] = L[l.name]["out"]
     chain = w8.w8a8_chain_create([L[l.name] for l in blk.layers])
     for _ in range(args.warmup):
@@ -829,10 +832,19 @@ def _run_block_on(args, blk, w8, rank, world, local, dev, stream) -> None:
     inst_ev = [[(torch.cuda.Event(enable_timing=True, external=True),
                  torch.cuda.Event(enable_timing=True, external=True)) for _ in blk.layers] for _ in range(R)]
 
+    def quantize(t):
+        q = w8.w8a8_quantize_act_gelu if t["input_act"] == w8.ACT_GELU else w8.w8a8_quantize_act
+        q(t["x"], xq=t["ws_xq"], scale_a=t["ws_scale_a"], stream=stream)
+
+    def linear(t):
+        f = w8.w8a8_linear_gelu if t["input_act"] == w8.ACT_GELU else w8.w8a8_linear
+        f(t["x"], t["wq"], t["scale_w"], t["bias"], out=t["out"], ws_xq=t["ws_xq"], ws_scale_a=t["ws_scale_a"],
+          stream=stream)
+
     def step_inst(i):
         for j, l in enumerate(blk.layers):
             t = L[l.name]
-            w8.w8a8_quantize_act(t["x"], xq=t["ws_xq"], scale_a=t["ws_scale_a"], stream=stream)
+            quantize(t)
             inst_ev[i][j][0].record(stream)
             w8.w8a8_gemm(t["ws_xq"], t["wq"], t["ws_scale_a"], t["scale_w"], t["bias"], out=t["out"], stream=stream)
             inst_ev[i][j][1].record(stream)
@@ -889,17 +901,25 @@ def _run_block_on(args, blk, w8, rank, world, local, dev, stream) -> None:
                      "larger than L2 except where noted)"}
     for l in blk.layers:
         t = L[l.name]
-        qms = graph_ms(lambda i, t=t: w8.w8a8_quantize_act(t["x"], xq=t["ws_xq"], scale_a=t["ws_scale_a"],
-                                                            stream=stream))
-        lms = graph_ms(lambda i, t=t: w8.w8a8_linear(t["x"], t["wq"], t["scale_w"], t["bias"], out=t["out"],
-                                                      ws_xq=t["ws_xq"], ws_scale_a=t["ws_scale_a"], stream=stream))
+        qms = graph_ms(lambda i, t=t: quantize(t))
+        lms = graph_ms(lambda i, t=t: linear(t))
         qbytes = 3 * M * l.K + 4 * M
         ops = 2.0 * M * l.N * l.K
-        comps[l.name] = {"N": l.N, "K": l.K, "gemm_ms_live": gemm_ms[l.name],
+        comps[l.name] = {"N": l.N, "K": l.K, "input_act": l.act or "none", "gemm_ms_live": gemm_ms[l.name],
                          "gemm_tops_live": ops / (gemm_ms[l.name] * 1e-3) / 1e12,
                          "linear_ms": lms, "quantizer_ms": qms, "quantizer_gbs": qbytes / (qms * 1e-3) / 1e9,
                          "quantizer_frac_of_measured_hbm": qbytes / (qms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                          "gemm_config": w8.w8a8_select_config(M, l.N, l.K)}
+        if l.act == "gelu":
+            # the same input unfused: a bf16 GELU kernel writes G, the quantizer reads it back
+            g = torch.empty_like(t["x"])
+            gms = graph_ms(lambda i, t=t, g=g: w8.w8a8_gelu(t["x"], g, stream=stream))
+            uqms = graph_ms(lambda i, t=t, g=g: w8.w8a8_quantize_act(g, xq=t["ws_xq"], scale_a=t["ws_scale_a"],
+                                                                        stream=stream))
+            comps[l.name]["unfused_gelu_ms"] = gms
+            comps[l.name]["unfused_quantizer_ms"] = uqms
+            comps[l.name]["fused_saves_ms"] = gms + uqms - qms
+            del g
     ctx = None
     if not args.no_context:
         bsrc = {"x": src["x"], "a": src["a"]}
@@ -907,8 +927,10 @@ def _run_block_on(args, blk, w8, rank, world, local, dev, stream) -> None:
 
         def bf16_block(i):
             for l in blk.layers:
-                torch.addmm(L[l.name]["bias"], bsrc[l.source] if l.source in bsrc else bout[l.source],
-                            wbf16[l.name].t(), out=bout[l.name])
+                xin = bsrc[l.source] if l.source in bsrc else bout[l.source]
+                if l.act == "gelu":
+                    xin = torch.nn.functional.gelu(xin, approximate="tanh")
+                torch.addmm(L[l.name]["bias"], xin, wbf16[l.name].t(), out=bout[l.name])
 
         for i in range(2):  # library handles are created outside graph capture
             bf16_block(i)

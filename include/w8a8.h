@@ -79,7 +79,8 @@ typedef enum {
 /* Human-readable name of a status code (static string, never NULL). */
 W8A8_API const char* w8a8_status_string(int status);
 
-/* ABI version of this header: 100 * major + minor. */
+/* ABI version of this header: 100 * major + minor (101: w8a8_linear_desc
+ * has input_act). */
 W8A8_API int w8a8_abi_version(void);
 
 /*
@@ -278,6 +279,36 @@ W8A8_API w8a8_status w8a8_linear_fp8(const void* x, const uint8_t* wq, const flo
                                      int64_t M, int64_t N, int64_t K, w8a8_stream_t stream);
 
 /*
+ * GELU before a linear layer, fused with its quantizer (the per-token
+ * quantizer moved into the producer of X: a DiT MLP's GELU sits between the
+ * up- and down-projections).  Unfused, a GELU kernel writes bf16 G =
+ * GELU(H) to HBM and the quantizer reads it back; fused, one pass reads H and
+ * writes the codes, saving a write and a read of G.  GELU is the tanh form
+ * (Hendrycks & Gimpel, "Gaussian Error Linear Units") written as
+ *   gelu(h) = h / (1 + exp(-2u)),  u = sqrt(2/pi) * (h + 0.044715 h^3),
+ * each step one binary32 operation in that order, exp the library's own
+ * (Cody-Waite reduction by ln 2 and a degree-7 Taylor polynomial, fused
+ * multiply-adds; +inf above 88, 0 below -30), rounded to bf16: exactly what
+ * w8a8_gelu stores.  The pages name no activation; this is the library's
+ * definition.
+ *
+ * w8a8_quantize_act_gelu: codes and scales of bf16_rne(gelu(h)); arguments
+ *   as w8a8_quantize_act (h in place of x).  Bit-identical to w8a8_gelu
+ *   followed by w8a8_quantize_act.
+ * w8a8_gelu: g = bf16_rne(gelu(h)), h and g bf16 [M, K] with row strides
+ *   ldh, ldg (multiples of 8 elements), K % 8 == 0.
+ * w8a8_linear_gelu: out = GELU(h) W^T + b through w8a8_quantize_act_gelu
+ *   and w8a8_gemm; arguments as w8a8_linear.
+ */
+W8A8_API w8a8_status w8a8_quantize_act_gelu(const void* h, int64_t M, int64_t K, int64_t ldh,
+                                            int8_t* xq, int64_t ldxq, float* scale_a, w8a8_stream_t stream);
+W8A8_API w8a8_status w8a8_gelu(const void* h, int64_t M, int64_t K, int64_t ldh, void* g, int64_t ldg,
+                               w8a8_stream_t stream);
+W8A8_API w8a8_status w8a8_linear_gelu(const void* h, const int8_t* wq, const float* scale_w, const void* bias,
+                                      void* out, int8_t* ws_xq, float* ws_scale_a,
+                                      int64_t M, int64_t N, int64_t K, w8a8_stream_t stream);
+
+/*
  * A chain of W8A8 linear layers as one CUDA graph (the paper drops its
  * kernel into every linear layer of the DiT, abstract; a DiT block runs
  * four: attention QKV, attention output, MLP up, MLP down).  Each layer is
@@ -294,6 +325,10 @@ W8A8_API w8a8_status w8a8_linear_fp8(const void* x, const uint8_t* wq, const flo
  * copies.  The chain holds no device memory.  Calls that launch the same
  * chain (or chains sharing buffers) must not overlap on the GPU.
  */
+/* Element-wise step a chain layer applies to its input before quantizing
+ * it (see w8a8_linear_gelu). */
+enum { W8A8_ACT_NONE = 0, W8A8_ACT_GELU = 1 };
+
 typedef struct {
     const void* x;            /* bf16 [M, K] input (row stride K) */
     const int8_t* wq;         /* int8 [N, K] weight codes */
@@ -303,6 +338,8 @@ typedef struct {
     int8_t* ws_xq;            /* int8 [M, K] workspace */
     float* ws_scale_a;        /* fp32 [M] workspace */
     int64_t M, N, K;
+    int32_t input_act;        /* W8A8_ACT_NONE, or W8A8_ACT_GELU: the layer computes GELU(x) W^T + b */
+    int32_t reserved;         /* zero */
 } w8a8_linear_desc;
 
 typedef struct w8a8_chain_st* w8a8_chain_t;

@@ -34,7 +34,7 @@ def test_status_strings(w8):
     for s in range(1, 7):
         assert w8.w8a8_status_string(s) not in ("ok", "unknown status")
     assert w8.w8a8_status_string(99) == "unknown status"
-    assert w8.w8a8_abi_version() == 100
+    assert w8.w8a8_abi_version() == 101
 
 
 def _gemm_i32(lib, xq, wq, acc, M, N, K):
@@ -92,6 +92,15 @@ def test_host_validation_without_device(w8):
     assert lib.w8a8_linear_fp8(A, A, A, None, A, A, None, 4, 8, 32, None) == 1    # no ws_scale_a
     cfg = w8.GemmConfig(block_m=256, block_n=256, stages=7, grid=2, raster_group=1)
     assert lib.w8a8_gemm_fp8_f32_ex(A, A, A, 4, 8, 32, ctypes.byref(cfg), None) == 1  # too many stages
+    # GELU before a linear layer
+    assert lib.w8a8_quantize_act_gelu(A, 4, 32, 16, A, 32, A, None) == 1    # ldx < K
+    assert lib.w8a8_quantize_act_gelu(A, 0, 32, 32, A, 32, A, None) == 0    # empty
+    assert lib.w8a8_gelu(A, 4, 12, 12, A, 12, None) == 1                    # K % 8
+    assert lib.w8a8_gelu(A, 4, 16, 20, A, 16, None) == 2                    # ldh % 8
+    assert lib.w8a8_gelu(A + 2, 4, 16, 16, A, 16, None) == 2                # misaligned h
+    assert lib.w8a8_gelu(A, 0, 16, 16, A, 16, None) == 0                    # empty
+    assert lib.w8a8_linear_gelu(A, A, A, None, A, A, A, 4, 12, 32, None) == 1
+    assert lib.w8a8_linear_gelu(A, A, A, None, A, A + 1, A, 4, 8, 32, None) == 2
     # chains of linear layers: every layer is validated before any CUDA call
     h = ctypes.c_void_p(None)
     assert lib.w8a8_chain_create(None, 1, ctypes.byref(h)) == 1
@@ -102,6 +111,8 @@ def test_host_validation_without_device(w8):
     d[1] = w8.LinearDesc(A, A, A, None, A, A + 4, A, 4, 8, 32)               # misaligned ws_xq
     assert lib.w8a8_chain_create(d, 2, ctypes.byref(h)) == 2 and not h.value
     assert lib.w8a8_chain_create(d, 0, ctypes.byref(h)) == 1
+    d[1] = w8.LinearDesc(A, A, A, None, A, A, A, 4, 8, 32, 7, 0)             # unknown input_act
+    assert lib.w8a8_chain_create(d, 2, ctypes.byref(h)) == 1
     assert lib.w8a8_chain_create(d, 1, None) == 1
     assert lib.w8a8_chain_launch(None, None) == 1
     assert lib.w8a8_chain_layers(None) == 0 and lib.w8a8_chain_destroy(None) == 0

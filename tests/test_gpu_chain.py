@@ -13,8 +13,8 @@ input for it, so whole chains are compared for equality, output by output
   (M = 9216): QKV 3072->9216 on the block input; attention output
   3072->3072 on a second input (the attention result, which is not part of
   this method); MLP up 3072->12288 on the attention output's result; MLP
-  down 12288->3072 on MLP up's result (the norm and GELU between them are
-  not part of this method either).  Weights quantized on the GPU are
+  down 12288->3072 on GELU of MLP up's result, the GELU fused into MLP
+  down's quantizer (the norm is not part of this method).  Weights quantized on the GPU are
   checked against the oracle's; the chain is checked on sampled rows (rows
   are independent through every layer)."""
 import numpy as np
@@ -101,11 +101,14 @@ def test_dit_block_1024_batch2(w8):
         wq_o, sw_o = oracle.quantize_weight(w)
         assert np.array_equal(wq.cpu().numpy(), wq_o) and np.array_equal(sw.cpu().numpy(), sw_o)
         b = d["bias_" + l.name]
-        L[l.name] = w8.linear_layer(src_t[l.source], wq, sw, bf16_bits_to_torch(b, dev))
+        act = w8.ACT_GELU if l.act == "gelu" else w8.ACT_NONE
+        L[l.name] = w8.linear_layer(src_t[l.source], wq, sw, bf16_bits_to_torch(b, dev), input_act=act)
         src_t[l.name] = L[l.name]["out"]
         # block inputs are sliced to the sampled rows; earlier layers' oracle
         # outputs already hold only those rows
         x_rows = src_o[l.source][rows] if l.source in ("x", "a") else src_o[l.source]
+        if l.act == "gelu":
+            x_rows = oracle.gelu(x_rows)
         ref[l.name] = _oracle_layer(x_rows, wq_o, sw_o, b)
         src_o[l.name] = ref[l.name][0]
     chain = w8.w8a8_chain_create([L[l.name] for l in blk.layers])

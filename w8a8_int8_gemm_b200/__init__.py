@@ -30,6 +30,7 @@ __all__ = [
     "w8a8_linear_noalloc",
     "w8a8_quantize_act_fp8", "w8a8_quantize_weight_fp8", "w8a8_gemm_fp8", "w8a8_gemm_fp8_ex",
     "w8a8_gemm_fp8_f32", "w8a8_gemm_fp8_f32_ex", "w8a8_linear_fp8",
+    "w8a8_quantize_act_gelu", "w8a8_gelu", "w8a8_linear_gelu", "ACT_NONE", "ACT_GELU",
     "LinearDesc", "Chain", "linear_layer", "w8a8_chain_create", "w8a8_chain_launch", "w8a8_chain_layers",
     "w8a8_chain_destroy",
     "w8a8_select_config",
@@ -42,6 +43,8 @@ header_path = os.path.join(os.path.dirname(_PKG), "include", "w8a8.h")
 
 W8A8_OK = 0
 W8A8_ERR_TIMEOUT = 5
+ACT_NONE = 0   # W8A8_ACT_NONE
+ACT_GELU = 1   # W8A8_ACT_GELU
 
 
 class W8A8Error(RuntimeError):
@@ -64,7 +67,7 @@ class LinearDesc(ctypes.Structure):
     _fields_ = [("x", ctypes.c_void_p), ("wq", ctypes.c_void_p), ("scale_w", ctypes.c_void_p),
                 ("bias", ctypes.c_void_p), ("out", ctypes.c_void_p), ("ws_xq", ctypes.c_void_p),
                 ("ws_scale_a", ctypes.c_void_p), ("M", ctypes.c_int64), ("N", ctypes.c_int64),
-                ("K", ctypes.c_int64)]
+                ("K", ctypes.c_int64), ("input_act", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 def _load() -> ctypes.CDLL:
@@ -94,6 +97,9 @@ def _load() -> ctypes.CDLL:
         "w8a8_gemm_fp8_f32": ([p, p, p, i64, i64, i64, p], ctypes.c_int),
         "w8a8_gemm_fp8_f32_ex": ([p, p, p, i64, i64, i64, ctypes.POINTER(GemmConfig), p], ctypes.c_int),
         "w8a8_linear_fp8": ([p, p, p, p, p, p, p, i64, i64, i64, p], ctypes.c_int),
+        "w8a8_quantize_act_gelu": ([p, i64, i64, i64, p, i64, p, p], ctypes.c_int),
+        "w8a8_gelu": ([p, i64, i64, i64, p, i64, p], ctypes.c_int),
+        "w8a8_linear_gelu": ([p, p, p, p, p, p, p, i64, i64, i64, p], ctypes.c_int),
         "w8a8_chain_create": ([ctypes.POINTER(LinearDesc), i32, ctypes.POINTER(p)], ctypes.c_int),
         "w8a8_chain_launch": ([p, p], ctypes.c_int),
         "w8a8_chain_layers": ([p], i32),
@@ -494,13 +500,57 @@ def w8a8_linear_fp8(x, wq, scale_w, bias=None, out=None, ws_xq=None, ws_scale_a=
     return out
 
 
+# ------------------------------------------------- GELU before a linear layer
+
+
+def w8a8_quantize_act_gelu(h, xq=None, scale_a=None, stream=None):
+    """Per-token int8 quantization of bf16_rne(GELU(h)) in one pass -> (xq int8 [M, K], scale_a fp32 [M])."""
+    _need(h, "h", torch.bfloat16, 2)
+    M, K = h.shape
+    if xq is None:
+        xq = torch.empty((M, K), dtype=torch.int8, device=h.device)
+    if scale_a is None:
+        scale_a = torch.empty((M,), dtype=torch.float32, device=h.device)
+    _need(xq, "xq", torch.int8, 2)
+    if tuple(xq.shape) != (M, K):
+        raise ValueError("xq must have the shape of h")
+    _need_contig(scale_a, "scale_a", torch.float32, (M,))
+    _check(_lib.w8a8_quantize_act_gelu(_ptr(h), M, K, h.stride(0) if M else K, _ptr(xq), xq.stride(0) if M else K,
+                                       _ptr(scale_a), _stream(stream, h.device)), "w8a8_quantize_act_gelu")
+    return xq, scale_a
+
+
+def w8a8_gelu(h, g=None, stream=None):
+    """g bf16 [M, K] = bf16_rne(GELU(h)) (the unfused producer)."""
+    _need(h, "h", torch.bfloat16, 2)
+    M, K = h.shape
+    if g is None:
+        g = torch.empty((M, K), dtype=torch.bfloat16, device=h.device)
+    _need(g, "g", torch.bfloat16, 2)
+    if tuple(g.shape) != (M, K):
+        raise ValueError("g must have the shape of h")
+    _check(_lib.w8a8_gelu(_ptr(h), M, K, h.stride(0) if M else K, _ptr(g), g.stride(0) if M else K,
+                          _stream(stream, h.device)), "w8a8_gelu")
+    return g
+
+
+def w8a8_linear_gelu(h, wq, scale_w, bias=None, out=None, ws_xq=None, ws_scale_a=None, stream=None):
+    """out bf16 [M, N] = GELU(h) W^T + b: w8a8_quantize_act_gelu then w8a8_gemm."""
+    l = linear_layer(h, wq, scale_w, bias, out, ws_xq, ws_scale_a, ACT_GELU)
+    _check(_lib.w8a8_linear_gelu(_ptr(l["x"]), _ptr(wq), _ptr(scale_w), _ptr(bias), _ptr(l["out"]),
+                                 _ptr(l["ws_xq"]), _ptr(l["ws_scale_a"]), l["M"], l["N"], l["K"],
+                                 _stream(stream, h.device)), "w8a8_linear_gelu")
+    return l["out"]
+
+
 # ------------------------------------------------- chains of linear layers
 
 
-def linear_layer(x, wq, scale_w, bias=None, out=None, ws_xq=None, ws_scale_a=None) -> dict:
+def linear_layer(x, wq, scale_w, bias=None, out=None, ws_xq=None, ws_scale_a=None, input_act: int = ACT_NONE) -> dict:
     """One layer of a chain: the tensors of a w8a8_linear call, with the
     output and workspace allocated here when not given.  x may be an
-    earlier layer's ``out``."""
+    earlier layer's ``out``; input_act=ACT_GELU makes the layer compute
+    GELU(x) W^T + b (w8a8_linear_gelu)."""
     _need(x, "x", torch.bfloat16, 2)
     M, K = x.shape
     _need(wq, "wq", torch.int8, 2)
@@ -520,7 +570,7 @@ def linear_layer(x, wq, scale_w, bias=None, out=None, ws_xq=None, ws_scale_a=Non
     _need_contig(ws_xq, "ws_xq", torch.int8, (M, K))
     _need_contig(ws_scale_a, "ws_scale_a", torch.float32, (M,))
     return {"x": x, "wq": wq, "scale_w": scale_w, "bias": bias, "out": out, "ws_xq": ws_xq,
-            "ws_scale_a": ws_scale_a, "M": M, "N": N, "K": K}
+            "ws_scale_a": ws_scale_a, "M": M, "N": N, "K": K, "input_act": int(input_act)}
 
 
 class Chain:
@@ -559,7 +609,8 @@ def w8a8_chain_create(layers: list) -> Chain:
     descs = (LinearDesc * max(1, len(layers)))()
     for i, l in enumerate(layers):
         descs[i] = LinearDesc(_ptr(l["x"]), _ptr(l["wq"]), _ptr(l["scale_w"]), _ptr(l.get("bias")), _ptr(l["out"]),
-                              _ptr(l["ws_xq"]), _ptr(l["ws_scale_a"]), l["M"], l["N"], l["K"])
+                              _ptr(l["ws_xq"]), _ptr(l["ws_scale_a"]), l["M"], l["N"], l["K"],
+                              int(l.get("input_act", ACT_NONE)), 0)
     h = ctypes.c_void_p(None)
     _check(_lib.w8a8_chain_create(descs, len(layers), ctypes.byref(h)), "w8a8_chain_create")
     return Chain(h.value, list(layers))

@@ -158,7 +158,7 @@ w8a8_status gemm_common(const int8_t* xq, const int8_t* wq, const float* scale_a
 }
 
 w8a8_status quantize_common(bool act, const void* x, int64_t M, int64_t K, int64_t ldx, int8_t* xq, int64_t ldxq,
-                            float* scale, cudaStream_t stream, bool e4m3 = false) {
+                            float* scale, cudaStream_t stream, bool e4m3 = false, bool gelu = false) {
   if (M < 0 || M > kMaxMN || K < 16 || K > kMaxK || K % 16 != 0) return W8A8_ERR_INVALID_ARG;
   if (ldx < K || ldxq < K) return W8A8_ERR_INVALID_ARG;
   if (M == 0) return W8A8_OK;
@@ -172,7 +172,9 @@ w8a8_status quantize_common(bool act, const void* x, int64_t M, int64_t K, int64
   const float* w = static_cast<const float*>(x);
   uint8_t* codes = reinterpret_cast<uint8_t*>(xq);
   cudaError_t e;
-  if (e4m3) {
+  if (gelu) {
+    e = launch_quantize_act_gelu(x, M, K, ldx, xq, ldxq, scale, stream);
+  } else if (e4m3) {
     e = act ? launch_quantize_act_e4m3(x, M, K, ldx, codes, ldxq, scale, stream)
             : launch_quantize_weight_e4m3(w, M, K, ldx, codes, ldxq, scale, stream);
   } else {
@@ -203,7 +205,7 @@ const char* w8a8_status_string(int status) {
   }
 }
 
-int w8a8_abi_version(void) { return 100; }
+int w8a8_abi_version(void) { return 101; }
 
 w8a8_status w8a8_quantize_act(const void* x, int64_t M, int64_t K, int64_t ldx, int8_t* xq, int64_t ldxq,
                               float* scale_a, w8a8_stream_t stream) {
@@ -355,6 +357,45 @@ w8a8_status w8a8_linear_fp8(const void* x, const uint8_t* wq, const float* scale
   return gemm_common(reinterpret_cast<const int8_t*>(ws_xq), reinterpret_cast<const int8_t*>(wq), ws_scale_a,
                      scale_w, bias, out, M, N, K, nullptr, GemmOut::kBf16Dequant,
                      reinterpret_cast<cudaStream_t>(stream), /*overlap_prologue=*/true, GemmElem::kE4M3);
+}
+
+// ------------------------------------------------- GELU before a linear layer
+
+w8a8_status w8a8_quantize_act_gelu(const void* h, int64_t M, int64_t K, int64_t ldh, int8_t* xq, int64_t ldxq,
+                                   float* scale_a, w8a8_stream_t stream) {
+  return quantize_common(true, h, M, K, ldh, xq, ldxq, scale_a, reinterpret_cast<cudaStream_t>(stream),
+                         /*e4m3=*/false, /*gelu=*/true);
+}
+
+w8a8_status w8a8_gelu(const void* h, int64_t M, int64_t K, int64_t ldh, void* g, int64_t ldg, w8a8_stream_t stream) {
+  if (M < 0 || M > kMaxMN || K < 8 || K > kMaxMN || K % 8 != 0 || ldh < K || ldg < K) return W8A8_ERR_INVALID_ARG;
+  if (M == 0) return W8A8_OK;
+  if (h == nullptr || g == nullptr) return W8A8_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(g) || ldh % 8 != 0 || ldg % 8 != 0) return W8A8_ERR_ALIGNMENT;
+  DeviceInfo dev;
+  w8a8_status st = current_device(&dev);
+  if (st != W8A8_OK) return st;
+  return from_cuda(launch_gelu(h, M, K, ldh, g, ldg, dev.sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+w8a8_status w8a8_linear_gelu(const void* h, const int8_t* wq, const float* scale_w, const void* bias, void* out,
+                             int8_t* ws_xq, float* ws_scale_a, int64_t M, int64_t N, int64_t K,
+                             w8a8_stream_t stream) {
+  w8a8_status st = check_gemm_shape(M, N, K);
+  if (st != W8A8_OK) return st;
+  if (M == 0 || N == 0) return W8A8_OK;
+  if (h == nullptr || wq == nullptr || scale_w == nullptr || out == nullptr || ws_xq == nullptr ||
+      ws_scale_a == nullptr) {
+    return W8A8_ERR_INVALID_ARG;
+  }
+  if (!aligned16(h) || !aligned16(wq) || !aligned16(scale_w) || !aligned16(bias) || !aligned16(out) ||
+      !aligned16(ws_xq) || !aligned16(ws_scale_a)) {
+    return W8A8_ERR_ALIGNMENT;
+  }
+  st = w8a8_quantize_act_gelu(h, M, K, K, ws_xq, K, ws_scale_a, stream);
+  if (st != W8A8_OK) return st;
+  return gemm_common(ws_xq, wq, ws_scale_a, scale_w, bias, out, M, N, K, nullptr, GemmOut::kBf16Dequant,
+                     reinterpret_cast<cudaStream_t>(stream), /*overlap_prologue=*/true);
 }
 
 int64_t w8a8_linear_sync_words(int64_t M) { return M < 0 ? 0 : linear_sync_words(M); }

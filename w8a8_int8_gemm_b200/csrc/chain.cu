@@ -12,8 +12,10 @@
 //
 // A layer's input may be an earlier layer's output (same buffer): the
 // graph keeps the stream order of the calls, so the later quantizer reads
-// the finished output.  The runner owns no device memory: every buffer is
-// the caller's and must outlive the chain.
+// the finished output.  A layer may apply GELU to its input on the way into
+// its quantizer (the producer of the input fused with the quantizer).  The
+// runner owns no device memory: every buffer is the caller's and must
+// outlive the chain.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -36,6 +38,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 w8a8_status check_layer(const w8a8_linear_desc& l) {
   if (l.M < 0 || l.N < 0 || l.K < 16 || l.K > 133144 || l.K % 16 != 0 || l.N % 8 != 0) return W8A8_ERR_INVALID_ARG;
   if (l.M > 2147483647 || l.N > 2147483647) return W8A8_ERR_INVALID_ARG;
+  if (l.input_act != W8A8_ACT_NONE && l.input_act != W8A8_ACT_GELU) return W8A8_ERR_INVALID_ARG;
   if (l.M == 0 || l.N == 0) return W8A8_OK;
   if (l.x == nullptr || l.wq == nullptr || l.scale_w == nullptr || l.out == nullptr || l.ws_xq == nullptr ||
       l.ws_scale_a == nullptr) {
@@ -79,8 +82,9 @@ w8a8_status w8a8_chain_create(const w8a8_linear_desc* layers, int32_t count, w8a
   }
   for (int32_t i = 0; i < count && st == W8A8_OK; ++i) {
     const w8a8_linear_desc& l = layers[i];
-    st = w8a8_linear(l.x, l.wq, l.scale_w, l.bias, l.out, l.ws_xq, l.ws_scale_a, l.M, l.N, l.K,
-                     reinterpret_cast<w8a8_stream_t>(s));
+    auto linear = l.input_act == W8A8_ACT_GELU ? w8a8_linear_gelu : w8a8_linear;
+    st = linear(l.x, l.wq, l.scale_w, l.bias, l.out, l.ws_xq, l.ws_scale_a, l.M, l.N, l.K,
+                reinterpret_cast<w8a8_stream_t>(s));
   }
   // Capture always ends, also after a failed layer (the partial graph is dropped).
   const cudaError_t ec = cudaStreamEndCapture(s, &graph);

@@ -60,6 +60,13 @@ cudaError_t launch_quantize_act_e4m3(const void* x, int64_t M, int64_t K, int64_
 cudaError_t launch_quantize_weight_e4m3(const float* w, int64_t N, int64_t K, int64_t ldw, uint8_t* q, int64_t ldq,
                                         float* scale, cudaStream_t stream);
 
+// GELU before a linear layer: the per-token quantizer applied to
+// bf16_rne(GELU(h)) in one pass, and the bf16 GELU alone.
+cudaError_t launch_quantize_act_gelu(const void* h, int64_t M, int64_t K, int64_t ldh, int8_t* q, int64_t ldq,
+                                     float* scale, cudaStream_t stream);
+cudaError_t launch_gelu(const void* h, int64_t M, int64_t K, int64_t ldh, void* g, int64_t ldg, int sms,
+                        cudaStream_t stream);
+
 // Largest stage count the shared memory holds for a tile shape (0 if none).
 // block_m 128: one CTA per tile; block_m 256: a CTA pair (cluster of 2).
 int gemm_max_stages(int block_m, int block_n);

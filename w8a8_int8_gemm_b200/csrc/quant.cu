@@ -49,6 +49,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 
 #include "internal.h"
@@ -61,7 +62,7 @@ namespace {
 // Rows of up to 32 * VPL vectors: the whole row in registers.  Seven
 // 128-thread blocks per SM (at most 72 registers) keep 28 rows per SM in
 // flight, so a 4096-token batch is resident in one wave on 148 SMs.
-template <typename T, int VPL, qrow::Code C>
+template <typename T, int VPL, qrow::Code C, qrow::Pre P>
 __global__ void __launch_bounds__(128, (VPL <= 12 ? 7 : 5))
     quantize_rows_regs_kernel(const T* __restrict__ x, int64_t M, int64_t K, int64_t ldx, int8_t* __restrict__ q,
                               int64_t ldq, float* __restrict__ scale) {
@@ -69,13 +70,13 @@ __global__ void __launch_bounds__(128, (VPL <= 12 ? 7 : 5))
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= M) return;
-  const float s = qrow::quantize_row<T, VPL, C>(reinterpret_cast<const uint4*>(x + row * ldx),
+  const float s = qrow::quantize_row<T, VPL, C, P>(reinterpret_cast<const uint4*>(x + row * ldx),
                                                 static_cast<int>(K / qrow::Vec<T>::kElems), q + row * ldq, lane);
   if (lane == 0) scale[row] = s;
 }
 
 // Any row length: absmax pass, then a second pass that reads the row again.
-template <typename T, qrow::Code C>
+template <typename T, qrow::Code C, qrow::Pre P>
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict__ x, int64_t M, int64_t K,
                                                             int64_t ldx, int8_t* __restrict__ q, int64_t ldq,
                                                             float* __restrict__ scale) {
@@ -83,14 +84,14 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict_
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= M) return;
-  const float s = qrow::quantize_row<T, 0, C>(reinterpret_cast<const uint4*>(x + row * ldx),
+  const float s = qrow::quantize_row<T, 0, C, P>(reinterpret_cast<const uint4*>(x + row * ldx),
                                               static_cast<int>(K / qrow::Vec<T>::kElems), q + row * ldq, lane);
   if (lane == 0) scale[row] = s;
 }
 
 // One 256-thread block per row of up to 256 * VPL vectors: the row in the
 // block's registers, |x| reduced over the block through shared memory.
-template <typename T, int VPL, qrow::Code C>
+template <typename T, int VPL, qrow::Code C, qrow::Pre P>
 __global__ void __launch_bounds__(256) quantize_rows_block_kernel(const T* __restrict__ x, int64_t K, int64_t ldx,
                                                                   int8_t* __restrict__ q, int64_t ldq,
                                                                   float* __restrict__ scale) {
@@ -107,7 +108,7 @@ __global__ void __launch_bounds__(256) quantize_rows_block_kernel(const T* __res
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int v = tid + 256 * i;
-    c[i] = v < nvec ? __ldg(xr + v) : make_uint4(0u, 0u, 0u, 0u);
+    c[i] = v < nvec ? qrow::pre_vec<T, P>(__ldg(xr + v)) : make_uint4(0u, 0u, 0u, 0u);
   }
   float amax = 0.0f;
 #pragma unroll
@@ -134,58 +135,89 @@ __global__ void __launch_bounds__(256) quantize_rows_block_kernel(const T* __res
   if (tid == 0) scale[row] = rs.s;
 }
 
-template <typename T, int VPL, qrow::Code C>
+template <typename T, int VPL, qrow::Code C, qrow::Pre P>
 void launch_regs(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq, float* scale,
                  cudaStream_t stream) {
   const int threads = 128;
   const int64_t blocks = (M + (threads / 32) - 1) / (threads / 32);
-  quantize_rows_regs_kernel<T, VPL, C>
+  quantize_rows_regs_kernel<T, VPL, C, P>
       <<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, M, K, ldx, q, ldq, scale);
 }
 
-template <typename T, int VPL, qrow::Code C>
+template <typename T, int VPL, qrow::Code C, qrow::Pre P>
 void launch_block(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq, float* scale,
                   cudaStream_t stream) {
-  quantize_rows_block_kernel<T, VPL, C><<<static_cast<unsigned>(M), 256, 0, stream>>>(x, K, ldx, q, ldq, scale);
+  quantize_rows_block_kernel<T, VPL, C, P><<<static_cast<unsigned>(M), 256, 0, stream>>>(x, K, ldx, q, ldq, scale);
 }
 
-template <typename T, qrow::Code C>
+template <typename T, qrow::Code C, qrow::Pre P = qrow::Pre::kNone>
 cudaError_t launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq, float* scale,
                             cudaStream_t stream) {
   const int64_t nvec = K / qrow::Vec<T>::kElems;
   const int64_t per_lane = (nvec + 31) / 32;
   if (per_lane <= 4) {
-    launch_regs<T, 4, C>(x, M, K, ldx, q, ldq, scale, stream);
+    launch_regs<T, 4, C, P>(x, M, K, ldx, q, ldq, scale, stream);
     return cudaGetLastError();
   }
   if (per_lane <= 8) {
-    launch_regs<T, 8, C>(x, M, K, ldx, q, ldq, scale, stream);
+    launch_regs<T, 8, C, P>(x, M, K, ldx, q, ldq, scale, stream);
     return cudaGetLastError();
   }
   if (per_lane <= 12) {
-    launch_regs<T, 12, C>(x, M, K, ldx, q, ldq, scale, stream);
+    launch_regs<T, 12, C, P>(x, M, K, ldx, q, ldq, scale, stream);
     return cudaGetLastError();
   }
   if (per_lane <= 16) {
-    launch_regs<T, 16, C>(x, M, K, ldx, q, ldq, scale, stream);
+    launch_regs<T, 16, C, P>(x, M, K, ldx, q, ldq, scale, stream);
     return cudaGetLastError();
   }
   const int64_t per_thread = (nvec + 255) / 256;  // one 256-thread block per row
   if (per_thread <= 8) {
-    launch_block<T, 8, C>(x, M, K, ldx, q, ldq, scale, stream);
+    launch_block<T, 8, C, P>(x, M, K, ldx, q, ldq, scale, stream);
   } else if (per_thread <= 12) {
-    launch_block<T, 12, C>(x, M, K, ldx, q, ldq, scale, stream);
+    launch_block<T, 12, C, P>(x, M, K, ldx, q, ldq, scale, stream);
   } else if (per_thread <= 16) {
-    launch_block<T, 16, C>(x, M, K, ldx, q, ldq, scale, stream);
+    launch_block<T, 16, C, P>(x, M, K, ldx, q, ldq, scale, stream);
   } else {
     const int threads = 256;
     const int64_t blocks = (M + (threads / 32) - 1) / (threads / 32);
-    quantize_rows_kernel<T, C><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, M, K, ldx, q, ldq, scale);
+    quantize_rows_kernel<T, C, P><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, M, K, ldx, q, ldq, scale);
   }
   return cudaGetLastError();
 }
 
+// bf16 GELU of rows h [M, K] into g: 16-byte vectors, grid-stride.
+__global__ void __launch_bounds__(256) gelu_rows_kernel(const __nv_bfloat16* __restrict__ h, int64_t M,
+                                                        int64_t K, int64_t ldh, __nv_bfloat16* __restrict__ g,
+                                                        int64_t ldg) {
+  const int64_t vpr = K / 8;  // vectors per row
+  const int64_t total = M * vpr;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / vpr;
+    const int64_t v = i - r * vpr;
+    const uint4 x = __ldg(reinterpret_cast<const uint4*>(h + r * ldh) + v);
+    reinterpret_cast<uint4*>(g + r * ldg)[v] = qrow::gelu_bf16x8(x);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_quantize_act_gelu(const void* h, int64_t M, int64_t K, int64_t ldh, int8_t* q, int64_t ldq,
+                                     float* scale, cudaStream_t stream) {
+  return launch_quantize<__nv_bfloat16, qrow::Code::kInt8, qrow::Pre::kGelu>(
+      static_cast<const __nv_bfloat16*>(h), M, K, ldh, q, ldq, scale, stream);
+}
+
+cudaError_t launch_gelu(const void* h, int64_t M, int64_t K, int64_t ldh, void* g, int64_t ldg, int sms,
+                        cudaStream_t stream) {
+  const int64_t total = M * (K / 8);
+  const int64_t max_blocks = static_cast<int64_t>(sms > 0 ? sms : 148) * 8;
+  const int64_t blocks = std::min<int64_t>(max_blocks, (total + 255) / 256);
+  gelu_rows_kernel<<<static_cast<unsigned>(blocks > 0 ? blocks : 1), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(h), M, K, ldh, static_cast<__nv_bfloat16*>(g), ldg);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq,
                                 float* scale, cudaStream_t stream) {

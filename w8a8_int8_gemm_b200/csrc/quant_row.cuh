@@ -19,6 +19,67 @@ namespace qrow {
 // Code format: int8 (scale absmax / 127) or E4M3 (scale absmax / 448).
 enum class Code { kInt8, kE4M3 };
 
+// Element-wise step applied to a bf16 row before it is quantized (the
+// producer of the linear layer's input, fused): none, or GELU.
+enum class Pre { kNone, kGelu };
+
+// exp(x) in binary32 as the library defines it: Cody-Waite reduction
+// x = k ln2 + r (ln2 split so that k * ln2_hi is exact), the degree-7 Taylor
+// polynomial of exp(r) by Horner's rule with fused multiply-adds, one product
+// with 2^k built from its bits; +inf above 88, 0 below -30.  Each step one
+// correctly rounded operation in this order (no approximate hardware
+// functions), so results are reproducible bit for bit off the GPU.
+__device__ __forceinline__ float own_expf(float x) {
+  if (x > 88.0f) return __int_as_float(0x7f800000);
+  if (x < -30.0f) return 0.0f;
+  const float k = rintf(__fmul_rn(x, 0x1.715476p+0f));  // log2 e
+  float r = __fmaf_rn(-k, 0x1.62e4p-1f, x);            // ln2, high part
+  r = __fmaf_rn(-k, 0x1.7f7d1cp-20f, r);               // ln2, low part
+  float p = 0x1.a01a02p-13f;                            // 1/5040
+  p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);                 // 1/720
+  p = __fmaf_rn(p, r, 0x1.111112p-7f);                  // 1/120
+  p = __fmaf_rn(p, r, 0x1.555556p-5f);                  // 1/24
+  p = __fmaf_rn(p, r, 0x1.555556p-3f);                  // 1/6
+  p = __fmaf_rn(p, r, 0.5f);
+  p = __fmaf_rn(p, r, 1.0f);
+  p = __fmaf_rn(p, r, 1.0f);
+  return __fmul_rn(p, __int_as_float((static_cast<int>(k) + 127) << 23));  // k in [-44, 127]
+}
+
+// GELU, tanh form (Hendrycks & Gimpel): h / (1 + exp(-2u)),
+// u = sqrt(2/pi) (h + 0.044715 h^3), one binary32 operation at a time.
+__device__ __forceinline__ float gelu_f32(float h) {
+  const float h3 = __fmul_rn(__fmul_rn(h, h), h);
+  const float inner = __fadd_rn(h, __fmul_rn(0x1.6e4e26p-5f, h3));  // 0.044715
+  const float u = __fmul_rn(0x1.988454p-1f, inner);                 // sqrt(2/pi)
+  const float e = own_expf(__fmul_rn(-2.0f, u));
+  return __fdiv_rn(h, __fadd_rn(1.0f, e));
+}
+
+// Eight bf16 -> bf16_rne(GELU) of each (what a GELU kernel would store).
+__device__ __forceinline__ uint4 gelu_bf16x8(const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = gelu_f32(__uint_as_float(w[i] << 16));
+    const float hi = gelu_f32(__uint_as_float(w[i] & 0xFFFF0000u));
+    const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+    o[i] = *reinterpret_cast<const uint32_t*>(&b);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+template <typename T, Pre P>
+__device__ __forceinline__ uint4 pre_vec(const uint4& v) {
+  if constexpr (P == Pre::kGelu) {
+    static_assert(sizeof(T) == 2, "GELU applies to bf16 activations");
+    return gelu_bf16x8(v);
+  } else {
+    return v;
+  }
+}
+
 template <Code C>
 __device__ __forceinline__ constexpr float code_max() {
   return C == Code::kInt8 ? 127.0f : 448.0f;
@@ -198,7 +259,7 @@ __device__ __forceinline__ void store_zero(int8_t* dst) {
 // the row's scale in every lane.  VPL > 0: rows of up to 32 * VPL vectors,
 // all loads issued at once and the row kept in registers; VPL == 0: any
 // length, an absmax pass and a second pass that reads the row again.
-template <typename T, int VPL, Code C = Code::kInt8>
+template <typename T, int VPL, Code C = Code::kInt8, Pre P = Pre::kNone>
 __device__ __forceinline__ float quantize_row(const uint4* __restrict__ xr, int nvec, int8_t* __restrict__ qr,
                                               int lane) {
   constexpr int E = Vec<T>::kElems;
@@ -207,7 +268,7 @@ __device__ __forceinline__ float quantize_row(const uint4* __restrict__ xr, int 
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int v = lane + 32 * i;
-      c[i] = v < nvec ? __ldg(xr + v) : make_uint4(0u, 0u, 0u, 0u);
+      c[i] = v < nvec ? pre_vec<T, P>(__ldg(xr + v)) : make_uint4(0u, 0u, 0u, 0u);
     }
     float amax = 0.0f;
 #pragma unroll
@@ -232,18 +293,18 @@ __device__ __forceinline__ float quantize_row(const uint4* __restrict__ xr, int 
     for (; v + 224 < nvec; v += 256) {
       uint4 a[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) a[i] = __ldg(xr + v + 32 * i);
+      for (int i = 0; i < 8; ++i) a[i] = pre_vec<T, P>(__ldg(xr + v + 32 * i));
 #pragma unroll
       for (int i = 0; i < 8; ++i) amax = fmaxf(amax, vec_absmax<T>(a[i]));
     }
-    for (; v < nvec; v += 32) amax = fmaxf(amax, vec_absmax<T>(__ldg(xr + v)));
+    for (; v < nvec; v += 32) amax = fmaxf(amax, vec_absmax<T>(pre_vec<T, P>(__ldg(xr + v))));
     const RowScale rs = row_scale<C>(amax);
     // pass 2: codes
     v = lane;
     for (; v + 96 < nvec; v += 128) {
       uint4 a[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = __ldg(xr + v + 32 * i);
+      for (int i = 0; i < 4; ++i) a[i] = pre_vec<T, P>(__ldg(xr + v + 32 * i));
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         if (rs.zero) {
@@ -257,7 +318,7 @@ __device__ __forceinline__ float quantize_row(const uint4* __restrict__ xr, int 
       if (rs.zero) {
         store_zero<E>(qr + E * v);
       } else {
-        encode_vec<T, C>(__ldg(xr + v), rs, qr + E * v);
+        encode_vec<T, C>(pre_vec<T, P>(__ldg(xr + v)), rs, qr + E * v);
       }
     }
     return rs.s;

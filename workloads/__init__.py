@@ -84,16 +84,17 @@ class BlockLayer:
     N: int
     K: int
     source: str           # "x" / "a": a block input; otherwise the name of the layer whose output feeds it
+    act: str = ""         # "gelu": the layer reads GELU(source), the GELU fused into its quantizer
 
 
 @dataclass(frozen=True)
 class Block:
     """The linear layers of one DiT block over M tokens, in execution order.
     Inputs "x" (the block input) and "a" (the attention result feeding the
-    attention output projection) are seeded bf16 N(0, 1); the norm,
-    attention and GELU between the linears are not part of the method, so
-    MLP up reads the attention output projection's result directly and MLP
-    down reads MLP up's."""
+    attention output projection) are seeded bf16 N(0, 1); the norm and the
+    attention are not part of the method, so MLP up reads the attention
+    output projection's result directly.  MLP down reads GELU of MLP up's
+    output, the GELU computed inside its quantizer."""
     name: str
     index: int
     M: int
@@ -124,7 +125,7 @@ class Block:
 BLOCKS: dict[str, Block] = {b.name: b for b in [
     Block("dit_block_1024", 6, 9216,
           (BlockLayer("qkv", 9216, 3072, "x"), BlockLayer("attn_out", 3072, 3072, "a"),
-           BlockLayer("mlp_up", 12288, 3072, "attn_out"), BlockLayer("mlp_down", 3072, 12288, "mlp_up")),
+           BlockLayer("mlp_up", 12288, 3072, "attn_out"), BlockLayer("mlp_down", 3072, 12288, "mlp_up", act="gelu")),
           note="the four linears of one DiT block, batch 2 at 1024px + 512 text tokens (M = 9216)"),
 ]}
 
