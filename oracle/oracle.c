@@ -41,7 +41,8 @@
  * GELU before a linear layer (the producer of its input, fused with the
  * per-token quantizer on the GPU): the tanh form h / (1 + exp(-2u)),
  * u = sqrt(2/pi) (h + 0.044715 h^3), with this file's own exp (Cody-Waite
- * reduction and a degree-7 Taylor polynomial), rounded to bf16:
+ * reduction and a degree-7 Taylor polynomial) and reciprocal (three
+ * Newton-Raphson steps), rounded to bf16:
  *
  *   g[r,k]    = bf16_rne( gelu(h[r,k]) ),  then the quantizer above on g
  *
@@ -229,9 +230,29 @@ float oracle_expf(float x) {
     return p * scale;
 }
 
+/* 1/d for 1 <= d <= 2^120, this library's own: an initial value from the
+ * bits of d (the integer 0x7EF311C3 - bits(d), within 12% of 1/d), two
+ * Newton-Raphson steps y <- y (2 - d y) (a fused multiply-add and a
+ * product each), then one in residual form y <- y + y (1 - d y) (two fused
+ * multiply-adds), which lands within an ulp of 1/d and on 1 exactly for
+ * d = 1. */
+static float oracle_recip(float d) {
+    uint32_t b;
+    memcpy(&b, &d, sizeof b);
+    uint32_t yb = 0x7EF311C3u - b;
+    float y;
+    memcpy(&y, &yb, sizeof y);
+    y = y * fmaf(-d, y, 2.0f);
+    y = y * fmaf(-d, y, 2.0f);
+    y = fmaf(y, fmaf(-d, y, 1.0f), y);
+    return y;
+}
+
 /* GELU, tanh form (Hendrycks & Gimpel, "Gaussian Error Linear Units"):
  * 0.5 h (1 + tanh(u)) = h / (1 + exp(-2u)), u = sqrt(2/pi) (h + 0.044715 h^3),
- * each operation rounded to binary32 in the order written. */
+ * each operation rounded to binary32 in the order written, the division
+ * taken as h times the reciprocal above; where -2u > 80 (|gelu| < 3e-34)
+ * the result is h * 0, a signed zero. */
 static const float GELU_C0 = 0.79788458347320556640625f;  /* fl32(sqrt(2 / pi)) */
 static const float GELU_C1 = 0.044715f;
 
@@ -239,8 +260,9 @@ float oracle_gelu_f32(float h) {
     float h3 = (h * h) * h;
     float inner = h + GELU_C1 * h3;
     float u = GELU_C0 * inner;
-    float e = oracle_expf(-2.0f * u);
-    return h / (1.0f + e);
+    float x = -2.0f * u;
+    if (x > 80.0f) return h * 0.0f;
+    return h * oracle_recip(1.0f + oracle_expf(x));
 }
 
 /* Element-wise over arrays (for the checks of these two functions). */

@@ -504,15 +504,16 @@ def _gelu_f64(h: np.ndarray) -> np.ndarray:
 def check_gelu_f32(orc) -> None:
     """GELU (tanh form) against the float64 formula h / (1 + exp(-2u)) within
     the binary32 error budget: u carries <= 7 roundings' relative error, which
-    exp turns into 14|u| ulp of relative error, plus 8 ulp for the rest; below
-    2^-122 in magnitude the cutoff of exp at 88 may give 0.  Closed forms:
-    gelu(0) = 0, gelu(h) = h exactly for h >= 10 (exp(-2u) < 2^-25), gelu(h)
-    = -0 for h <= -13 (exp argument above 88)."""
+    exp turns into 14|u| ulp of relative error, plus 12 ulp for exp, the sum,
+    the Newton reciprocal and the product; below 2^-110 in magnitude the
+    cutoff (-2u > 80 gives a signed zero) may give 0.  Closed forms:
+    gelu(0) = 0, gelu(h) = h exactly for h >= 10 (exp(-2u) < 2^-25, and the
+    reciprocal of 1 is 1), gelu(h) = -0 for h <= -13."""
     h = np.concatenate([np.linspace(-20, 20, 400001), np.linspace(-1e-3, 1e-3, 20001),
                         np.geomspace(1e-30, 1e4, 20000), -np.geomspace(1e-30, 1e4, 20000)]).astype(np.float32)
     g = orc.gelu_f32(h).astype(np.float64)
     gt, u = _gelu_f64(h)
-    bound = (14 * np.abs(u) + 8) * 2.0 ** -24 * np.abs(gt) + 2.0 ** -122
+    bound = (14 * np.abs(u) + 12) * 2.0 ** -24 * np.abs(gt) + 2.0 ** -110
     assert (np.abs(g - gt) <= bound).all(), float((np.abs(g - gt) / bound).max())
     big = np.linspace(10, 3e38, 1001).astype(np.float32)
     assert np.array_equal(orc.gelu_f32(big), big)

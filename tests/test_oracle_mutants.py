@@ -55,8 +55,11 @@ MUTANTS = [
     ("gelu cubic coefficient 0.04471", "static const float GELU_C1 = 0.044715f;",
      "static const float GELU_C1 = 0.04471f;"),
     ("gelu without the cubic term", "float inner = h + GELU_C1 * h3;", "float inner = h;"),
-    ("gelu wrong sign in exp", "float e = oracle_expf(-2.0f * u);", "float e = oracle_expf(2.0f * u);"),
-    ("gelu 1 - e", "return h / (1.0f + e);", "return h / (1.0f - e);"),
+    ("gelu wrong sign in exp", "float x = -2.0f * u;", "float x = 2.0f * u;"),
+    ("gelu 1 - e", "oracle_recip(1.0f + oracle_expf(x))", "oracle_recip(1.0f - oracle_expf(x))"),
+    ("reciprocal without the residual step", "    y = fmaf(y, fmaf(-d, y, 1.0f), y);\n", ""),
+    ("reciprocal initial value a factor 4 off", "uint32_t yb = 0x7EF311C3u - b;",
+     "uint32_t yb = 0x7DF311C3u - b;"),
     ("exp without the low part of ln2", "r = fmaf(-k, LN2_LO, r);", ""),
     ("exp Taylor term r^7 dropped", "float p = 1.0f / 5040.0f;", "float p = 0.0f;"),
     ("exp scale off by one", "uint32_t bits = (uint32_t)((int32_t)k + 127) << 23;",
