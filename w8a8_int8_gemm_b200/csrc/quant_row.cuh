@@ -23,37 +23,90 @@ enum class Code { kInt8, kE4M3 };
 // producer of the linear layer's input, fused): none, or GELU.
 enum class Pre { kNone, kGelu };
 
-// exp(x) in binary32 as the library defines it: Cody-Waite reduction
-// x = k ln2 + r (ln2 split so that k * ln2_hi is exact), the degree-7 Taylor
-// polynomial of exp(r) by Horner's rule with fused multiply-adds, one product
-// with 2^k built from its bits; +inf above 88, 0 below -30.  Each step one
-// correctly rounded operation in this order (no approximate hardware
-// functions), so results are reproducible bit for bit off the GPU.
-__device__ __forceinline__ float own_expf(float x) {
-  if (x > 88.0f) return __int_as_float(0x7f800000);
-  if (x < -30.0f) return 0.0f;
-  const float k = rintf(__fmul_rn(x, 0x1.715476p+0f));  // log2 e
-  float r = __fmaf_rn(-k, 0x1.62e4p-1f, x);            // ln2, high part
-  r = __fmaf_rn(-k, 0x1.7f7d1cp-20f, r);               // ln2, low part
-  float p = 0x1.a01a02p-13f;                            // 1/5040
-  p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);                 // 1/720
-  p = __fmaf_rn(p, r, 0x1.111112p-7f);                  // 1/120
-  p = __fmaf_rn(p, r, 0x1.555556p-5f);                  // 1/24
-  p = __fmaf_rn(p, r, 0x1.555556p-3f);                  // 1/6
-  p = __fmaf_rn(p, r, 0.5f);
-  p = __fmaf_rn(p, r, 1.0f);
-  p = __fmaf_rn(p, r, 1.0f);
-  return __fmul_rn(p, __int_as_float((static_cast<int>(k) + 127) << 23));  // k in [-44, 127]
+// Packed binary32 pairs (Blackwell f32x2 arithmetic): each lane of the
+// pair is rounded exactly as the scalar operation would round it.
+namespace f2 {
+__device__ __forceinline__ uint64_t pack(float lo, float hi) {
+  uint64_t v;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
+  return v;
 }
+__device__ __forceinline__ void unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t splat(float x) { return pack(x, x); }
+__device__ __forceinline__ uint64_t fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t neg(uint64_t a) { return a ^ 0x8000000080000000ull; }
+}  // namespace f2
 
-// GELU, tanh form (Hendrycks & Gimpel): h / (1 + exp(-2u)),
-// u = sqrt(2/pi) (h + 0.044715 h^3), one binary32 operation at a time.
-__device__ __forceinline__ float gelu_f32(float h) {
-  const float h3 = __fmul_rn(__fmul_rn(h, h), h);
-  const float inner = __fadd_rn(h, __fmul_rn(0x1.6e4e26p-5f, h3));  // 0.044715
-  const float u = __fmul_rn(0x1.988454p-1f, inner);                 // sqrt(2/pi)
-  const float e = own_expf(__fmul_rn(-2.0f, u));
-  return __fdiv_rn(h, __fadd_rn(1.0f, e));
+// GELU of two binary32 values, as the library defines it: the tanh form
+// (Hendrycks & Gimpel) h / (1 + exp(-2u)), u = sqrt(2/pi) (h + 0.044715 h^3),
+// each step one correctly rounded binary32 operation in this order (the
+// pair's lanes computed together by packed instructions):
+//   * exp(x), x = -2u, the library's own: Cody-Waite reduction x = k ln2 + r
+//     (ln2 split so that k * ln2_hi is exact), the degree-7 Taylor polynomial
+//     of exp(r) by Horner's rule with fused multiply-adds, one product with
+//     2^k built from its bits; 0 below -30 (it is evaluated at -30 there and
+//     discarded);
+//   * the division as h times the library's reciprocal of d = 1 + exp(x): an
+//     initial value from the bits of d (0x7EF311C3 - bits(d)), two
+//     Newton-Raphson steps y (2 - d y), one residual step y + y (1 - d y);
+//   * where x > 80 the result is h * 0, a signed zero.
+// No approximate hardware function is used, so the result is reproducible
+// bit for bit off the GPU.
+__device__ __forceinline__ void gelu_f32x2(float& a, float& b) {
+  const uint64_t h = f2::pack(a, b);
+  const uint64_t h3 = f2::mul(f2::mul(h, h), h);
+  const uint64_t inner = f2::add(h, f2::mul(f2::splat(0x1.6e4e26p-5f), h3));  // 0.044715
+  const uint64_t u = f2::mul(f2::splat(0x1.988454p-1f), inner);                // sqrt(2/pi)
+  float x0, x1;
+  f2::unpack(f2::mul(f2::splat(-2.0f), u), x0, x1);
+  const uint64_t xc = f2::pack(fminf(fmaxf(x0, -30.0f), 80.0f), fminf(fmaxf(x1, -30.0f), 80.0f));
+  float t0, t1;
+  f2::unpack(f2::mul(xc, f2::splat(0x1.715476p+0f)), t0, t1);  // log2 e
+  const float k0 = rintf(t0), k1 = rintf(t1);
+  const uint64_t nk = f2::pack(-k0, -k1);
+  uint64_t r = f2::fma(nk, f2::splat(0x1.62e4p-1f), xc);    // ln2, high part
+  r = f2::fma(nk, f2::splat(0x1.7f7d1cp-20f), r);           // ln2, low part
+  uint64_t p = f2::splat(0x1.a01a02p-13f);                  // 1/5040
+  p = f2::fma(p, r, f2::splat(0x1.6c16c2p-10f));            // 1/720
+  p = f2::fma(p, r, f2::splat(0x1.111112p-7f));             // 1/120
+  p = f2::fma(p, r, f2::splat(0x1.555556p-5f));             // 1/24
+  p = f2::fma(p, r, f2::splat(0x1.555556p-3f));             // 1/6
+  p = f2::fma(p, r, f2::splat(0.5f));
+  p = f2::fma(p, r, f2::splat(1.0f));
+  p = f2::fma(p, r, f2::splat(1.0f));
+  float e0, e1;
+  f2::unpack(f2::mul(p, f2::pack(__int_as_float((static_cast<int>(k0) + 127) << 23),
+                                 __int_as_float((static_cast<int>(k1) + 127) << 23))),
+             e0, e1);
+  const uint64_t d = f2::add(f2::splat(1.0f), f2::pack(x0 < -30.0f ? 0.0f : e0, x1 < -30.0f ? 0.0f : e1));
+  float d0, d1;
+  f2::unpack(d, d0, d1);
+  uint64_t y = f2::pack(__uint_as_float(0x7EF311C3u - __float_as_uint(d0)),
+                        __uint_as_float(0x7EF311C3u - __float_as_uint(d1)));
+  const uint64_t nd = f2::neg(d);
+  y = f2::mul(y, f2::fma(nd, y, f2::splat(2.0f)));
+  y = f2::mul(y, f2::fma(nd, y, f2::splat(2.0f)));
+  y = f2::fma(y, f2::fma(nd, y, f2::splat(1.0f)), y);
+  float g0, g1;
+  f2::unpack(f2::mul(h, y), g0, g1);
+  a = x0 > 80.0f ? __fmul_rn(a, 0.0f) : g0;
+  b = x1 > 80.0f ? __fmul_rn(b, 0.0f) : g1;
 }
 
 // Eight bf16 -> bf16_rne(GELU) of each (what a GELU kernel would store).
@@ -62,8 +115,9 @@ __device__ __forceinline__ uint4 gelu_bf16x8(const uint4& v) {
   uint32_t o[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float lo = gelu_f32(__uint_as_float(w[i] << 16));
-    const float hi = gelu_f32(__uint_as_float(w[i] & 0xFFFF0000u));
+    float lo = __uint_as_float(w[i] << 16);
+    float hi = __uint_as_float(w[i] & 0xFFFF0000u);
+    gelu_f32x2(lo, hi);
     const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
     o[i] = *reinterpret_cast<const uint32_t*>(&b);
   }
