@@ -336,6 +336,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    // Every operand load of this CTA is issued: a kernel launched as this
+    // one's programmatic dependent may be scheduled (it waits for this
+    // grid's completion before reading anything it writes).
+    pdl_launch_dependents();
     if (!ok && PAIR && lane == 0) st_cluster_u32(peer_abort, 1u);
     // Teardown: the last fill of each stage must have landed before the CTA
     // exits (on the normal path the MMA warp already waited for all of

@@ -66,7 +66,12 @@ template <typename T, int VPL, qrow::Code C, qrow::Pre P>
 __global__ void __launch_bounds__(128, (VPL <= 12 ? 7 : 5))
     quantize_rows_regs_kernel(const T* __restrict__ x, int64_t M, int64_t K, int64_t ldx, int8_t* __restrict__ q,
                               int64_t ldq, float* __restrict__ scale) {
-  pdl_launch_dependents();  // a GEMM launched after this may be scheduled already
+  // Launched as a programmatic dependent of the kernel before it (whose
+  // output may be x): wait for that kernel first, then let this kernel's own
+  // dependent (the GEMM, which reads its weight operand before it waits) be
+  // scheduled.
+  pdl_wait_prerequisites();
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= M) return;
@@ -80,6 +85,11 @@ template <typename T, qrow::Code C, qrow::Pre P>
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const T* __restrict__ x, int64_t M, int64_t K,
                                                             int64_t ldx, int8_t* __restrict__ q, int64_t ldq,
                                                             float* __restrict__ scale) {
+  // Launched as a programmatic dependent of the kernel before it (whose
+  // output may be x): wait for that kernel first, then let this kernel's own
+  // dependent (the GEMM, which reads its weight operand before it waits) be
+  // scheduled.
+  pdl_wait_prerequisites();
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -95,6 +105,11 @@ template <typename T, int VPL, qrow::Code C, qrow::Pre P>
 __global__ void __launch_bounds__(256) quantize_rows_block_kernel(const T* __restrict__ x, int64_t K, int64_t ldx,
                                                                   int8_t* __restrict__ q, int64_t ldq,
                                                                   float* __restrict__ scale) {
+  // Launched as a programmatic dependent of the kernel before it (whose
+  // output may be x): wait for that kernel first, then let this kernel's own
+  // dependent (the GEMM, which reads its weight operand before it waits) be
+  // scheduled.
+  pdl_wait_prerequisites();
   pdl_launch_dependents();
   constexpr int E = qrow::Vec<T>::kElems;
   constexpr int kWarps = 8;
@@ -135,19 +150,39 @@ __global__ void __launch_bounds__(256) quantize_rows_block_kernel(const T* __res
   if (tid == 0) scale[row] = rs.s;
 }
 
+// Launch as a programmatic dependent of the previous kernel in the stream:
+// the launch overlaps that kernel's tail, and the kernel's first act is to
+// wait for it (griddepcontrol.wait).
+template <typename... Params, typename... Args>
+void launch_after_prev(void (*kernel)(Params...), unsigned blocks, unsigned threads, cudaStream_t stream,
+                       Args... args) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(blocks);
+  lc.blockDim = dim3(threads);
+  lc.dynamicSmemBytes = 0;
+  lc.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  cudaLaunchKernelEx(&lc, kernel, static_cast<Params>(args)...);
+}
+
 template <typename T, int VPL, qrow::Code C, qrow::Pre P>
 void launch_regs(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq, float* scale,
                  cudaStream_t stream) {
   const int threads = 128;
   const int64_t blocks = (M + (threads / 32) - 1) / (threads / 32);
-  quantize_rows_regs_kernel<T, VPL, C, P>
-      <<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, M, K, ldx, q, ldq, scale);
+  launch_after_prev(quantize_rows_regs_kernel<T, VPL, C, P>, static_cast<unsigned>(blocks), threads, stream, x, M,
+                    K, ldx, q, ldq, scale);
 }
 
 template <typename T, int VPL, qrow::Code C, qrow::Pre P>
 void launch_block(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq, float* scale,
                   cudaStream_t stream) {
-  quantize_rows_block_kernel<T, VPL, C, P><<<static_cast<unsigned>(M), 256, 0, stream>>>(x, K, ldx, q, ldq, scale);
+  launch_after_prev(quantize_rows_block_kernel<T, VPL, C, P>, static_cast<unsigned>(M), 256, stream, x, K, ldx,
+                    q, ldq, scale);
 }
 
 template <typename T, qrow::Code C, qrow::Pre P = qrow::Pre::kNone>
@@ -181,7 +216,8 @@ cudaError_t launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_
   } else {
     const int threads = 256;
     const int64_t blocks = (M + (threads / 32) - 1) / (threads / 32);
-    quantize_rows_kernel<T, C, P><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, M, K, ldx, q, ldq, scale);
+    launch_after_prev(quantize_rows_kernel<T, C, P>, static_cast<unsigned>(blocks), threads, stream, x, M, K, ldx,
+                      q, ldq, scale);
   }
   return cudaGetLastError();
 }
