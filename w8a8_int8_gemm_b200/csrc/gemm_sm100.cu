@@ -9,24 +9,32 @@
 // The paper's kernel is Triton on Ampere mma.sync; this one is written for
 // the 5th-generation tensor cores:
 //
-//   * persistent: one CTA per SM walks output tiles of BLOCK_M x BLOCK_N
-//     (128 x 256 or 128 x 128) in a grouped raster order;
-//   * warp 0 (one elected lane) streams K-slices of 128 bytes of both
+//   * persistent: one CTA (or CTA pair) per SM (pair of SMs) walks output
+//     tiles of BLOCK_M x BLOCK_N in a grouped raster order; when the last
+//     round would leave at least half of them idle, its tiles run as two
+//     half-width items each;
+//   * tiles: 128 x 256 or 128 x 128 on one CTA, or 256 x 256 / 256 x 128 on
+//     a CTA pair (tcgen05 cta_group::2: each CTA loads its 128 rows of A and
+//     half of B, the leader issues M=256 MMAs over both CTAs' shared memory,
+//     each CTA's tensor memory holds its 128 rows of the accumulator);
+//   * warp 0 (one elected lane) streams K-chunks of 128 bytes of both
 //     operands with TMA into a ring of shared-memory stages (128-byte
-//     swizzle), signalling "full" mbarriers with transaction counts;
+//     swizzle), signalling "full" mbarriers with transaction counts; a
+//     pair's stage holds two K-chunks loaded as one box each through 3-D
+//     tensor maps when K allows (larger requests: the per-SM TMA delivery
+//     rate depends on them);
 //   * warp 1 allocates tensor memory and (one elected lane) issues
-//     tcgen05.mma.kind::i8, M=128, N=BLOCK_N, K=32 per instruction, into
-//     int32 accumulators held in tensor memory; tcgen05.commit frees each
-//     ring stage when its MMAs retire and marks the accumulator full after
-//     the last K-slice;
-//   * warps 2-5 (the epilogue) each own one 32-lane quarter of tensor
-//     memory (= 32 output rows): they load the int32 accumulators, apply
-//     the dequantization and bias in binary32 in the order above, round to
-//     bf16, stage 32 x 64 bf16 blocks in swizzled shared memory and write
-//     them with TMA stores;
+//     tcgen05.mma.kind::i8, K=32 per instruction, into int32 accumulators
+//     held in tensor memory; tcgen05.commit frees each ring stage when its
+//     MMAs retire and marks the accumulator full after the last K-chunk;
+//   * warps 2-9 (the epilogue) work two per 32-lane quarter of tensor
+//     memory (= 32 output rows), each on half of the tile's columns: they
+//     load the int32 accumulators, apply the dequantization and bias in
+//     binary32 in the order above, round to bf16, stage 32 x 64 bf16 blocks
+//     in swizzled shared memory and write them with TMA stores;
 //   * the accumulator is double-buffered in tensor memory (2 x BLOCK_N
 //     columns), so the epilogue of one tile overlaps the MMAs of the next.
-//
+
 // The same kernel runs the FP8 variant (OCP E4M3 operands, the paper's
 // comparison baseline): tcgen05.mma.kind::f8f6f4, also K=32 bytes per
 // instruction, so the tiles, the ring and the swizzle are unchanged; the
