@@ -452,6 +452,19 @@ def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
         side["linear_ms"] = graph_ms(step_linear, max(3, 300 // G))
         if not fp8:
             side["fused_ms"] = graph_ms(step_fused, max(3, 300 // G))
+        # the floor for the quantizer's byte count: a plain device copy moving
+        # the same bytes (half read, half written), same harness, same rotation
+        half = quant_bytes // 2 // 16 * 16
+        copy_src = [torch.empty(half, dtype=torch.uint8, device=dev) for _ in range(nsets)]
+        copy_dst = [torch.empty(half, dtype=torch.uint8, device=dev) for _ in range(nsets)]
+        for t in copy_src:
+            t.fill_(1)
+
+        def step_copy(i):
+            copy_dst[i % nsets].copy_(copy_src[i % nsets])
+
+        side["copy_ms"] = graph_ms(step_copy, max(3, 300 // G))
+        del copy_src, copy_dst
         side = {k: v for k, v in side.items() if v is not None}
     traffic = ncu_traffic(wl.name, "fp8" if fp8 else args.path)
 
@@ -503,6 +516,12 @@ def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
                 result["components"]["quantizer"] = {"ms": side["quant_ms"], "gbs": qg,
                                                      "frac_of_measured_hbm": qg / peaks["hbm_gbs"],
                                                      "frac_of_8tbs": qg / 8000.0, "bytes": quant_bytes}
+                if "copy_ms" in side:
+                    cg = 2 * (quant_bytes // 2 // 16 * 16) / (side["copy_ms"] * 1e-3) / 1e9
+                    result["components"]["quantizer"]["copy_floor"] = {
+                        "ms": side["copy_ms"], "gbs": cg, "frac_of_measured_hbm": cg / peaks["hbm_gbs"],
+                        "what": "torch copy_ moving the quantizer's byte count (half read, half written), "
+                                "graph of back-to-back calls over rotating buffers"}
             for key, name in (("gemm_ms", gemm.__name__), ("linear_ms", linear.__name__),
                               ("fused_ms", "w8a8_linear_fused")):
                 if key in side:

@@ -1,0 +1,35 @@
+"""bench.py's reference arm on the CPU: it runs the oracle on a bounded
+sample and prints one JSON line with the keys the benchmark contract asks
+for (the native arm needs a GPU and is exercised by the GPU runs)."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+KEYS = {"impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+        "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e", "gpu_launches"}
+
+
+@pytest.mark.parametrize("args", [["--workload", "tiny"], ["--workload", "tiny", "--format", "fp8"],
+                                  ["--workload", "dit_block_1024"]], ids=["int8", "fp8", "block"])
+def test_reference_arm_json(args):
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "3", "--warmup", "3"]
+    out = subprocess.run(cmd + args, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1, out.stdout
+    d = json.loads(lines[0])
+    assert KEYS <= set(d), KEYS - set(d)
+    assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 3 and d["warmup"] == 3
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["gpu_launches"] == 0
+
+
+def test_warmup_below_three_is_rejected():
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+           "--steps", "3", "--warmup", "2"]
+    out = subprocess.run(cmd, capture_output=True, text=True, timeout=120, cwd=ROOT)
+    assert out.returncode != 0
