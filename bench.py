@@ -454,14 +454,16 @@ def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
             side["fused_ms"] = graph_ms(step_fused, max(3, 300 // G))
         # the floor for the quantizer's byte count: a plain device copy moving
         # the same bytes (half read, half written), same harness, same rotation
+        # (its own rotation, combined footprint > 3x L2, so that it is HBM traffic)
         half = quant_bytes // 2 // 16 * 16
-        copy_src = [torch.empty(half, dtype=torch.uint8, device=dev) for _ in range(nsets)]
-        copy_dst = [torch.empty(half, dtype=torch.uint8, device=dev) for _ in range(nsets)]
+        ncopy = max(2, int(np.ceil(3 * L2_BYTES / (2 * half))))
+        copy_src = [torch.empty(half, dtype=torch.uint8, device=dev) for _ in range(ncopy)]
+        copy_dst = [torch.empty(half, dtype=torch.uint8, device=dev) for _ in range(ncopy)]
         for t in copy_src:
             t.fill_(1)
 
         def step_copy(i):
-            copy_dst[i % nsets].copy_(copy_src[i % nsets])
+            copy_dst[i % ncopy].copy_(copy_src[i % ncopy])
 
         side["copy_ms"] = graph_ms(step_copy, max(3, 300 // G))
         del copy_src, copy_dst
@@ -521,7 +523,7 @@ def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
                     result["components"]["quantizer"]["copy_floor"] = {
                         "ms": side["copy_ms"], "gbs": cg, "frac_of_measured_hbm": cg / peaks["hbm_gbs"],
                         "what": "torch copy_ moving the quantizer's byte count (half read, half written), "
-                                "graph of back-to-back calls over rotating buffers"}
+                                "graph of back-to-back calls over rotating buffers larger than 3x L2"}
             for key, name in (("gemm_ms", gemm.__name__), ("linear_ms", linear.__name__),
                               ("fused_ms", "w8a8_linear_fused")):
                 if key in side:
