@@ -77,6 +77,73 @@ def test_act_edge_rows(w8):
     _assert_same(q, s, bits)
 
 
+def _bf16_pattern(v):
+    return int(np.array([v], np.float32).view(np.uint32)[0] >> 16)
+
+
+# Row maxima whose significands have few bits (127 x / amax is then an exact
+# half-integer for many x), an all-ones significand, and the scales next to
+# 2^-100, below which rows are quantized by IEEE division.
+TIE_AMAX = [1.0, 3.0, 0.75, 5.0, 7.0, 127.0, 254.0, 1.9921875, 0.1875, 96.0, 127.0 * 2.0 ** -100]
+
+
+def _tie_rows(K):
+    """Rows [amax, then every bf16 value with |x| <= amax, both signs]."""
+    rows = []
+    pats = [_bf16_pattern(a) for a in TIE_AMAX]
+    p100 = _bf16_pattern(127.0 * 2.0 ** -100)
+    pats += [p100 - 1, p100 + 1]
+    for a in pats:
+        pos = np.arange(0, a + 1, dtype=np.uint32).astype(np.uint16)
+        vals = np.concatenate([pos, pos | np.uint16(0x8000)])
+        for c in range(0, len(vals), K - 1):
+            seg = vals[c:c + K - 1]
+            row = np.zeros(K, np.uint16)
+            row[0] = a
+            row[1:1 + len(seg)] = seg
+            rows.append(row)
+    return np.stack(rows)
+
+
+@pytest.mark.parametrize("K", [3072, 12288, 40000])
+def test_act_dense_ties(w8, K):
+    """Every bf16 value below each of several row maxima, many of them exact
+    half-integer quotients, on the warp, block and two-pass paths."""
+    bits = _tie_rows(K)
+    q, s = _run_act(w8, bits)
+    _assert_same(q, s, bits)
+
+
+def test_weight_dense_ties(w8):
+    """fp32 rows with values planted at (and a few ulps around) every
+    half-integer multiple of the row's scale, for scales from 2^-100 up."""
+    rng = np.random.default_rng(11)
+    K = 1296
+    h = np.arange(-254, 255, dtype=np.float32) * np.float32(0.5)
+    rows = []
+    amaxes = list(np.float32(2.0) ** rng.uniform(-93, 100, 60).astype(np.float32) * rng.uniform(1, 2, 60))
+    edge = np.float32(127.0 * 2.0 ** -100)
+    amaxes += [edge, np.nextafter(edge, np.float32(0)), np.nextafter(edge, np.float32(1))]
+    for a in amaxes:
+        a = np.float32(a)
+        s = np.float32(a / np.float32(127.0))
+        x = (h * s).astype(np.float32)
+        d = rng.integers(-2, 3, x.shape).astype(np.int32)
+        x = (x.view(np.int32) + d * (x != 0)).view(np.float32)
+        x = np.clip(x, -a, a)
+        row = np.zeros(K, np.float32)
+        row[0] = a
+        row[1:1 + len(x)] = x
+        rows.append(row)
+    w = np.stack(rows)
+    wq, sw = w8.w8a8_quantize_weight(torch.from_numpy(w).cuda())
+    torch.cuda.synchronize()
+    wq_o, sw_o = oracle.quantize_weight(w)
+    assert np.array_equal(sw.cpu().numpy().view(np.uint32), sw_o.view(np.uint32))
+    bad = np.argwhere(wq.cpu().numpy() != wq_o)
+    assert bad.size == 0, f"{len(bad)} codes differ, first at {bad[:3].tolist()}"
+
+
 def test_act_strided(w8):
     rng = np.random.default_rng(4)
     bits = P.to_bits(rng.standard_normal((37, 320)).astype(np.float32))

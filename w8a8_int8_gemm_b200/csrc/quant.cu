@@ -21,31 +21,31 @@
 // bf16 element (2 in, 1 out): the kernels are bound by HBM bandwidth.
 //
 // Exactness.  The code q is decided in binary32 exactly as the definition
-// says.  Instead of one IEEE division per element, the kernel multiplies by
-// the row's reciprocal r = fl32(1/scale) and only divides where that could
-// change the rounded integer.  With |x/scale| <= 127 (1 + 2^-23), the exact
-// product t = x*r differs from the exact quotient x/scale by at most
-// 127.0001 * 2^-24 < 2^-17, and fl32(x/scale) differs from x/scale by at
-// most 2^-18, so rne(t) == rne(fl32(x/scale)) unless t lies within 2^-16 of
-// a half-integer.  t is rounded to an integer by a fused multiply-add with
-// 1.5 * 2^23 (one rounding of x*r + 1.5*2^23, to nearest even); the low byte
-// of the result's bit pattern is then the two's-complement int8 code, and
-// |t| <= 127.0001 keeps it inside [-127, 127] without a clamp.  A second
-// fused multiply-add gives the residual t - rne(t) (error <= 2^-25); a
-// vector holding an element whose residual is within 2^-15 of +-0.5 is redone
-// with IEEE division (__fdiv_rn) in an out-of-line path.  Rows whose scale is
-// not a normal number, or whose reciprocal is not finite, take the division
-// for every element.
+// says, without one IEEE division per element: the quotient fl32(x/scale) is
+// formed from the row's reciprocal r = fl32(1/scale) by Markstein's
+// correction (q0 = fl32(x*r); the remainder x - q0*scale is exact in one
+// fused multiply-add; fl32(q0 + remainder*r) is the correctly rounded
+// quotient), three packed f32x2 operations per element pair, and rounded to
+// an integer by adding 1.5*2^23 (ties to even), whose bit pattern's low byte
+// is the int8 code.  An earlier scheme rounded the bare product x*r and
+// redid near-half-integer elements by division; bf16 rows defeat it: with
+// both x and amax bf16, 127*x/amax is an exact half-integer for about 0.3%
+// of the elements of N(0,1) rows, one warp step in four, and the redo cost
+// a third of the kernel's time.  The correction was checked against IEEE
+// division for every pair of bf16 values |x| <= amax and on 10^9 planted
+// fp32 elements.  Rows whose scale is below 2^-100 (where the remainder can
+// underflow), or whose reciprocal is not finite, take IEEE division
+// (__fdiv_rn) for every element.
 //
 // FP8 variant (OCP E4M3 codes; B200's native FP8 path, the comparison
 // baseline of the same paper): the same scheme with 448, the largest finite
 // E4M3 value, in place of 127:
 //   scale[r] = fl32(max_k |x[r,k]| / 448)
 //   q[r,k]   = e4m3_rne(clamp(fl32(x[r,k] / scale[r]), -448, 448)), 0 if scale[r] == 0
-// Each element takes one IEEE division and one hardware conversion
-// (cvt.rn.satfinite.e4m3x2.f32: round to nearest even, saturating), which is
-// the definition term by term; a negative quotient that rounds to zero keeps
-// its sign (code 0x80).
+// Each element's quotient is the same correctly rounded fl32(x/scale) (with
+// x's sign, so that a negative quotient that rounds to zero keeps it: code
+// 0x80), then one hardware conversion (cvt.rn.satfinite.e4m3x2.f32: round to
+// nearest even, saturating), which is the definition term by term.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 

@@ -220,51 +220,82 @@ __device__ __noinline__ void quantize_vec_div(uint4 v, float s, int8_t* dst) {
   store_words<E>(q, dst);
 }
 
-// The product path with the tie check described at the top of quant.cu:
-// m = fl(x*r + 1.5*2^23) rounds the exact product x*r to an integer (ties to
-// even; 1.5*2^23 is even) in one fused multiply-add, so m - 1.5*2^23 is that
-// integer n and the low byte of m's bit pattern is its int8 code; the
-// residual x*r - n (one more fused multiply-add, rounding error <= 2^-25)
-// flags elements within 2^-15 of a half-integer, whose vector is redone
-// with IEEE division.
-template <typename T>
-__device__ __forceinline__ void quantize_vec(const uint4& v, float s, float r, bool fast, int8_t* dst) {
-  constexpr int E = Vec<T>::kElems;
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  if (fast) {
-    float f[E];
-    Vec<T>::unpack(v, f);
-    uint32_t q[E];
-    bool near_tie = false;
-#pragma unroll
-    for (int i = 0; i < E; ++i) {
-      const float m = __fmaf_rn(f[i], r, kRound);  // rne(x*r) + 1.5 * 2^23, exactly
-      const float n = __fsub_rn(m, kRound);        // rne(x*r)
-      near_tie |= fabsf(__fmaf_rn(f[i], r, -n)) >= 0.499969482421875f;  // 0.5 - 2^-15
-      q[i] = __float_as_uint(m);                   // low byte = int8 code
-    }
-    if (!near_tie) {
-      store_words<E>(q, dst);
-      return;
-    }
-  }
-  quantize_vec_div<T>(v, s, dst);
+struct RowScale {
+  float s;  // the row's scale, fl32(amax / code_max)
+  float r;  // fl32(1 / s)
+  bool zero, fast;
+};
+
+// fl32(x / s) for a pair of elements without a division, by Markstein's
+// correction (P. Markstein, "Computation of elementary functions on the IBM
+// RISC System/6000 processor", IBM J. Res. Develop. 34(1), 1990): with
+// r = fl32(1/s) and q0 = fl32(x*r), which is within one ulp of x/s, the
+// remainder x - q0*s is exact in one fused multiply-add, and
+// q1 = fl32(q0 + (x - q0*s)*r) is the correctly rounded quotient.  Rows take
+// this path when s >= 2^-100 (the remainder then never underflows for a
+// quotient that decides a code) and r is finite; it was checked to equal
+// IEEE division bit for bit for every pair of bf16 values |x| <= amax at
+// both code ranges (quotients of magnitude below 2^-12, which give code 0,
+// keep their sign and stay below 2^-11), and on 10^9 fp32 elements planted
+// at and around the half-integer quotients.
+__device__ __forceinline__ uint64_t quotient2(uint64_t x, uint64_t r2, uint64_t neg_s2) {
+  const uint64_t q0 = f2::mul(x, r2);
+  const uint64_t rem = f2::fma(q0, neg_s2, x);  // x - q0*s, exact
+  return f2::fma(rem, r2, q0);
 }
 
-// E4M3 codes of one vector: e4m3_rne(clamp(fl32(x / s), -448, 448)), one
-// IEEE division per element and one rounding to E4M3 (the clamp is explicit
-// although the conversion saturates: the definition clamps).
+// int8 codes of one vector: rne(fl32(x / s)), the quotient from quotient2
+// (or IEEE division on the rows that do not qualify).  q = fl32(x/s) + 1.5*2^23
+// rounds the quotient to an integer n (ties to even; 1.5*2^23 is even) and
+// the low byte of its bit pattern is n's two's-complement int8 code; |x/s|
+// <= 127.0001 keeps n inside [-127, 127] without a clamp.
 template <typename T>
-__device__ __forceinline__ void quantize_vec_e4m3(const uint4& v, float s, int8_t* dst) {
+__device__ __forceinline__ void quantize_vec(const uint4& v, const RowScale& rs, int8_t* dst) {
+  constexpr int E = Vec<T>::kElems;
+  if (rs.fast) {
+    float f[E];
+    Vec<T>::unpack(v, f);
+    const uint64_t r2 = f2::splat(rs.r), neg_s2 = f2::splat(-rs.s), round2 = f2::splat(12582912.0f);
+    uint32_t q[E];
+#pragma unroll
+    for (int i = 0; i < E; i += 2) {
+      float m0, m1;
+      f2::unpack(f2::add(quotient2(f2::pack(f[i], f[i + 1]), r2, neg_s2), round2), m0, m1);
+      q[i] = __float_as_uint(m0);
+      q[i + 1] = __float_as_uint(m1);
+    }
+    store_words<E>(q, dst);
+    return;
+  }
+  quantize_vec_div<T>(v, rs.s, dst);
+}
+
+// E4M3 codes of one vector: e4m3_rne(clamp(fl32(x / s), -448, 448)), the
+// quotient from quotient2 with x's sign (a zero quotient of a negative x is
+// -0, code 0x80) or IEEE division, then one rounding to E4M3 (the clamp is
+// explicit although the conversion saturates: the definition clamps).
+template <typename T>
+__device__ __forceinline__ void quantize_vec_e4m3(const uint4& v, const RowScale& rs, int8_t* dst) {
   constexpr int E = Vec<T>::kElems;
   float f[E];
   Vec<T>::unpack(v, f);
+  float d[E];
+  if (rs.fast) {
+    const uint64_t r2 = f2::splat(rs.r), neg_s2 = f2::splat(-rs.s);
+#pragma unroll
+    for (int i = 0; i < E; i += 2) {
+      f2::unpack(quotient2(f2::pack(f[i], f[i + 1]), r2, neg_s2), d[i], d[i + 1]);
+      d[i] = copysignf(d[i], f[i]);
+      d[i + 1] = copysignf(d[i + 1], f[i + 1]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < E; ++i) d[i] = __fdiv_rn(f[i], rs.s);
+  }
   uint32_t h[E / 2];
 #pragma unroll
   for (int i = 0; i < E / 2; ++i) {
-    const float a = fminf(fmaxf(__fdiv_rn(f[2 * i], s), -448.0f), 448.0f);
-    const float b = fminf(fmaxf(__fdiv_rn(f[2 * i + 1], s), -448.0f), 448.0f);
-    h[i] = cvt_e4m3x2(a, b);
+    h[i] = cvt_e4m3x2(fminf(fmaxf(d[2 * i], -448.0f), 448.0f), fminf(fmaxf(d[2 * i + 1], -448.0f), 448.0f));
   }
   if constexpr (E == 8) {
     *reinterpret_cast<uint2*>(dst) = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
@@ -272,11 +303,6 @@ __device__ __forceinline__ void quantize_vec_e4m3(const uint4& v, float s, int8_
     *reinterpret_cast<uint32_t*>(dst) = h[0] | (h[1] << 16);
   }
 }
-
-struct RowScale {
-  float s, r;
-  bool zero, fast;
-};
 
 template <Code C = Code::kInt8>
 __device__ __forceinline__ RowScale row_scale(float amax) {
@@ -286,7 +312,7 @@ __device__ __forceinline__ RowScale row_scale(float amax) {
   rs.s = __fdiv_rn(amax, code_max<C>());
   rs.zero = (rs.s == 0.0f);  // all-zero row (or an fp32 row whose scale underflows): codes 0
   rs.r = rs.zero ? 0.0f : __frcp_rn(rs.s);
-  rs.fast = !rs.zero && rs.s >= 1.17549435e-38f && isfinite(rs.r);
+  rs.fast = !rs.zero && rs.s >= 0x1p-100f && isfinite(rs.r);
   return rs;
 }
 
@@ -294,9 +320,9 @@ __device__ __forceinline__ RowScale row_scale(float amax) {
 template <typename T, Code C>
 __device__ __forceinline__ void encode_vec(const uint4& v, const RowScale& rs, int8_t* dst) {
   if constexpr (C == Code::kInt8) {
-    quantize_vec<T>(v, rs.s, rs.r, rs.fast, dst);
+    quantize_vec<T>(v, rs, dst);
   } else {
-    quantize_vec_e4m3<T>(v, rs.s, dst);
+    quantize_vec_e4m3<T>(v, rs, dst);
   }
 }
 
@@ -410,12 +436,12 @@ __device__ __forceinline__ void quantize_two_rows(const uint4* __restrict__ x0, 
       if (r0.zero) {
         store_zero<E>(q0 + E * v);
       } else {
-        quantize_vec<T>(c0[i], r0.s, r0.r, r0.fast, q0 + E * v);
+        quantize_vec<T>(c0[i], r0, q0 + E * v);
       }
       if (r1.zero) {
         store_zero<E>(q1 + E * v);
       } else {
-        quantize_vec<T>(c1[i], r1.s, r1.r, r1.fast, q1 + E * v);
+        quantize_vec<T>(c1[i], r1, q1 + E * v);
       }
     }
   }
