@@ -22,6 +22,7 @@
 #include <new>
 
 #include "../../include/w8a8.h"
+#include "internal.h"
 
 struct w8a8_chain_st {
   cudaGraph_t graph = nullptr;
@@ -74,6 +75,13 @@ w8a8_status w8a8_chain_create(const w8a8_linear_desc* layers, int32_t count, w8a
 
   cudaStream_t s = nullptr;
   if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return W8A8_ERR_CUDA;
+  for (int32_t i = 0; i < count; ++i) {
+    if (layers[i].input_act == W8A8_ACT_GELU && layers[i].M > 0 && layers[i].N > 0 &&
+        w8a8::prepare_quantize_act_gelu(layers[i].K, s) != cudaSuccess) {
+      cudaStreamDestroy(s);
+      return W8A8_ERR_CUDA;
+    }
+  }
   w8a8_status st = W8A8_OK;
   cudaGraph_t graph = nullptr;
   if (cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {

@@ -66,6 +66,9 @@ cudaError_t launch_quantize_act_gelu(const void* h, int64_t M, int64_t K, int64_
                                      float* scale, cudaStream_t stream);
 cudaError_t launch_gelu(const void* h, int64_t M, int64_t K, int64_t ldh, void* g, int64_t ldg, int sms,
                         cudaStream_t stream);
+// Kernel setup for launch_quantize_act_gelu on rows of K, made before a
+// stream capture that will record it.
+cudaError_t prepare_quantize_act_gelu(int64_t K, cudaStream_t stream);
 
 // Largest stage count the shared memory holds for a tile shape (0 if none).
 // block_m 128: one CTA per tile; block_m 256: a CTA pair (cluster of 2).

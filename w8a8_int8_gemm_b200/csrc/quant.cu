@@ -16,7 +16,9 @@
 // 256-thread block (K <= 32768 bf16, 16384 fp32): one block per row, the row
 // in the block's registers, |x| reduced across its warps through shared
 // memory, one pass over HBM.  Longer still: a two-pass register kernel that
-// reads the row twice.  |x| is reduced with butterfly shuffles; the codes are
+// reads the row twice.  GELU before the quantizer (and the bf16 GELU alone)
+// goes through a table of GELU over all 65536 bf16 inputs in shared memory
+// for rows of up to 16384 (see the table kernels below).  |x| is reduced with butterfly shuffles; the codes are
 // written packed (8 or 4 bytes per lane per vector).  HBM sees 3 bytes per
 // bf16 element (2 in, 1 out): the kernels are bound by HBM bandwidth.
 //
@@ -51,6 +53,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <mutex>
 
 #include "internal.h"
 #include "quant_row.cuh"
@@ -222,10 +225,135 @@ cudaError_t launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_
   return cudaGetLastError();
 }
 
-// bf16 GELU of rows h [M, K] into g: 16-byte vectors, grid-stride.
-__global__ void __launch_bounds__(256) gelu_rows_kernel(const __nv_bfloat16* __restrict__ h, int64_t M,
-                                                        int64_t K, int64_t ldh, __nv_bfloat16* __restrict__ g,
-                                                        int64_t ldg) {
+// ---------------------------------------------------------------------------
+// GELU fused into the per-token quantizer, by table.  GELU's input is bf16,
+// so it takes one of 65536 values, and what the quantizer consumes,
+// bf16_rne(GELU(h)), is a function of the 16 input bits alone.  The kernel
+// evaluates that function for every bit pattern with the same packed
+// arithmetic the other kernels apply element by element (gelu_bf16x8), into
+// a 128 KB table in shared memory, and then replaces the ~31 instructions of
+// GELU per element by one shared-memory load.  The table is built by a
+// cluster of CTAs: each computes 65536 / cluster entries and stores them into
+// the shared memory of every CTA of the cluster (distributed shared memory),
+// then the cluster synchronises once.  This happens before the kernel waits
+// for its producer, so it overlaps the tail of the kernel that writes h.
+//
+// Rows: a persistent grid of one 1024-thread CTA per SM; each 256-thread
+// group (four per CTA) quantizes one row at a time, VPL 16-byte vectors per
+// thread held in registers, |GELU(h)| reduced over the group's eight warps
+// through shared memory and a named barrier.
+constexpr int kLutGroups = 4;
+constexpr int kLutThreads = 256 * kLutGroups;
+constexpr int kLutTableBytes = 65536 * 2;
+constexpr int kLutSmemBytes = kLutTableBytes + 2 * kLutGroups * 8 * 4;
+
+__device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, const uint4& v) {
+  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Two bf16 of a word -> their table entries, packed the same way.  The pack
+// is an opaque prmt so that the row stays four registers per vector (seen
+// through, the compiler keeps every entry in a register of its own and the
+// row no longer fits the 64 registers a thread has at 1024 threads).
+__device__ __forceinline__ uint32_t lut_pair(const uint16_t* table, uint32_t w) {
+  const uint32_t lo = table[w & 0xFFFFu];
+  const uint32_t hi = table[w >> 16];
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+
+// The table of bf16_rne(GELU(h)) for every bf16 bit pattern h, built by a
+// cluster: this CTA computes 65536 / cluster consecutive entries (8 per
+// packed evaluation) and stores each 16-byte run into the table of every CTA
+// of the cluster.  The caller synchronises the cluster before any lookup.
+__device__ __forceinline__ void build_gelu_table(uint16_t* table, int cluster) {
+  const uint32_t rank = cluster_ctarank();
+  const int per_cta = 65536 / cluster;
+  const uint32_t table_addr = smem_u32(table);
+  for (int e = static_cast<int>(rank) * per_cta + static_cast<int>(threadIdx.x) * 8;
+       e < static_cast<int>(rank + 1) * per_cta; e += static_cast<int>(blockDim.x) * 8) {
+    const uint32_t u = static_cast<uint32_t>(e);
+    const uint4 pats = make_uint4(u | ((u + 1) << 16), (u + 2) | ((u + 3) << 16), (u + 4) | ((u + 5) << 16),
+                                  (u + 6) | ((u + 7) << 16));
+    const uint4 g = qrow::gelu_bf16x8(pats);
+    for (int r = 0; r < cluster; ++r) st_cluster_v4(map_to_cta(table_addr + 2u * u, static_cast<uint32_t>(r)), g);
+  }
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(kLutThreads, 1)
+    quantize_rows_gelu_lut_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t K, int64_t ldx,
+                                  int8_t* __restrict__ q, int64_t ldq, float* __restrict__ scale, int cluster) {
+  extern __shared__ __align__(16) uint8_t lut_smem[];
+  uint16_t* table = reinterpret_cast<uint16_t*>(lut_smem);
+  float* wmax = reinterpret_cast<float*>(lut_smem + kLutTableBytes);  // [2][kLutGroups][8]
+  const int tid = threadIdx.x;
+  build_gelu_table(table, cluster);
+  // h is the previous kernel's output: wait for it only now.
+  pdl_wait_prerequisites();
+  pdl_launch_dependents();
+  cluster_sync_all();  // every table entry written and visible; no remote access after this
+
+  const int grp = tid >> 8;
+  const int t = tid & 255;
+  const int lane = tid & 31;
+  const int warp = t >> 5;
+  const int nvec = static_cast<int>(K / 8);
+  int parity = 0;
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * kLutGroups + grp; row < M;
+       row += static_cast<int64_t>(gridDim.x) * kLutGroups, parity ^= 1) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * ldx);
+    uint4 c[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int v = t + 256 * i;
+      c[i] = v < nvec ? __ldg(xr + v) : make_uint4(0u, 0u, 0u, 0u);  // GELU(+0) = +0
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      c[i] = make_uint4(lut_pair(table, c[i].x), lut_pair(table, c[i].y), lut_pair(table, c[i].z),
+                        lut_pair(table, c[i].w));
+      amax = fmaxf(amax, qrow::vec_absmax<__nv_bfloat16>(c[i]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    float* slot = wmax + (parity * kLutGroups + grp) * 8;
+    if (lane == 0) slot[warp] = amax;
+    named_barrier_sync(1 + grp, 256);
+#pragma unroll
+    for (int w = 0; w < 8; ++w) amax = fmaxf(amax, slot[w]);
+    const qrow::RowScale rs = qrow::row_scale<qrow::Code::kInt8>(amax);
+    int8_t* qr = q + row * ldq;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int v = t + 256 * i;
+      if (v < nvec) {
+        if (rs.zero) {
+          qrow::store_zero<8>(qr + 8 * v);
+        } else {
+          qrow::encode_vec<__nv_bfloat16, qrow::Code::kInt8>(c[i], rs, qr + 8 * v);
+        }
+      }
+    }
+    if (t == 0) scale[row] = rs.s;
+  }
+}
+
+// bf16 GELU of rows h [M, K] into g by the same table: a persistent grid
+// over the rows' 16-byte vectors, eight lookups per vector.
+__global__ void __launch_bounds__(kLutThreads, 1)
+    gelu_rows_lut_kernel(const __nv_bfloat16* __restrict__ h, int64_t M, int64_t K, int64_t ldh,
+                         __nv_bfloat16* __restrict__ g, int64_t ldg, int cluster) {
+  extern __shared__ __align__(16) uint8_t lut_smem[];
+  uint16_t* table = reinterpret_cast<uint16_t*>(lut_smem);
+  build_gelu_table(table, cluster);
+  pdl_wait_prerequisites();
+  pdl_launch_dependents();
+  cluster_sync_all();
   const int64_t vpr = K / 8;  // vectors per row
   const int64_t total = M * vpr;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
@@ -233,26 +361,147 @@ __global__ void __launch_bounds__(256) gelu_rows_kernel(const __nv_bfloat16* __r
     const int64_t r = i / vpr;
     const int64_t v = i - r * vpr;
     const uint4 x = __ldg(reinterpret_cast<const uint4*>(h + r * ldh) + v);
-    reinterpret_cast<uint4*>(g + r * ldg)[v] = qrow::gelu_bf16x8(x);
+    reinterpret_cast<uint4*>(g + r * ldg)[v] =
+        make_uint4(lut_pair(table, x.x), lut_pair(table, x.y), lut_pair(table, x.z), lut_pair(table, x.w));
   }
+}
+
+// Launch geometry of the table kernels on one device: cluster size and the
+// number of clusters that are resident at once (one CTA per SM).
+struct LutGeometry {
+  int cluster = 0;
+  int clusters = 0;
+};
+
+template <auto kernel>
+LutGeometry lut_geometry(cudaStream_t stream) {
+  constexpr int kMaxDev = 64;
+  static std::mutex mu;
+  static LutGeometry cache[kMaxDev];  // one per kernel (template argument) and device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev].cluster != 0) return cache[dev];
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutSmemBytes) != cudaSuccess) {
+    return {};
+  }
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 2) return {};
+  // Clusters of 2 always fit side by side (SMs come in pairs); larger ones
+  // are taken when the occupancy query says that at least as many SMs stay
+  // busy.  The query is not made while the stream is being captured.
+  LutGeometry g{2, sms / 2};
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusNone) {
+    for (int c : {8, 4}) {
+      cudaLaunchConfig_t lc = {};
+      lc.gridDim = dim3(c * (sms / c));
+      lc.blockDim = dim3(kLutThreads);
+      lc.dynamicSmemBytes = kLutSmemBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = c;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      lc.attrs = attr;
+      lc.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kernel, &lc) == cudaSuccess && n * c >= 2 * (sms / 2) - 8) {
+        g = LutGeometry{c, n};
+        break;
+      }
+      (void)cudaGetLastError();
+    }
+    cache[dev] = g;
+  }
+  return g;
+}
+
+template <int VPL>
+cudaError_t launch_gelu_lut(const __nv_bfloat16* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq,
+                            float* scale, cudaStream_t stream) {
+  const LutGeometry g = lut_geometry<quantize_rows_gelu_lut_kernel<VPL>>(stream);
+  if (g.cluster == 0) return cudaErrorInvalidConfiguration;
+  const int64_t rows_per_cluster = static_cast<int64_t>(kLutGroups) * g.cluster;
+  const int64_t clusters = std::min<int64_t>(g.clusters, (M + rows_per_cluster - 1) / rows_per_cluster);
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(static_cast<unsigned>(clusters * g.cluster));
+  lc.blockDim = dim3(kLutThreads);
+  lc.dynamicSmemBytes = kLutSmemBytes;
+  lc.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(g.cluster);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 2;
+  return cudaLaunchKernelEx(&lc, quantize_rows_gelu_lut_kernel<VPL>, x, M, K, ldx, q, ldq, scale, g.cluster);
 }
 
 }  // namespace
 
+// Sets up the table kernel that launch_quantize_act_gelu uses for rows of K
+// (its shared-memory size and cluster geometry) outside of any stream
+// capture, so that a captured launch gets the geometry chosen by the
+// occupancy query rather than the fallback.
+cudaError_t prepare_quantize_act_gelu(int64_t K, cudaStream_t stream) {
+  const int64_t per_thread = (K / 8 + 255) / 256;
+  LutGeometry g;
+  if (per_thread <= 2) {
+    g = lut_geometry<quantize_rows_gelu_lut_kernel<2>>(stream);
+  } else if (per_thread <= 4) {
+    g = lut_geometry<quantize_rows_gelu_lut_kernel<4>>(stream);
+  } else if (per_thread <= 6) {
+    g = lut_geometry<quantize_rows_gelu_lut_kernel<6>>(stream);
+  } else if (per_thread <= 8) {
+    g = lut_geometry<quantize_rows_gelu_lut_kernel<8>>(stream);
+  } else {
+    return cudaSuccess;  // longer rows use the row kernels, which need no setup
+  }
+  return g.cluster != 0 ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
+// GELU then per-token int8 codes: rows of up to 16384 bf16 through the table
+// kernel, longer rows through the row kernels with GELU evaluated per
+// element (both give the same bits).
 cudaError_t launch_quantize_act_gelu(const void* h, int64_t M, int64_t K, int64_t ldh, int8_t* q, int64_t ldq,
                                      float* scale, cudaStream_t stream) {
-  return launch_quantize<__nv_bfloat16, qrow::Code::kInt8, qrow::Pre::kGelu>(
-      static_cast<const __nv_bfloat16*>(h), M, K, ldh, q, ldq, scale, stream);
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(h);
+  const int64_t per_thread = (K / 8 + 255) / 256;
+  if (per_thread <= 2) return launch_gelu_lut<2>(x, M, K, ldh, q, ldq, scale, stream);
+  if (per_thread <= 4) return launch_gelu_lut<4>(x, M, K, ldh, q, ldq, scale, stream);
+  if (per_thread <= 6) return launch_gelu_lut<6>(x, M, K, ldh, q, ldq, scale, stream);
+  if (per_thread <= 8) return launch_gelu_lut<8>(x, M, K, ldh, q, ldq, scale, stream);
+  return launch_quantize<__nv_bfloat16, qrow::Code::kInt8, qrow::Pre::kGelu>(x, M, K, ldh, q, ldq, scale, stream);
 }
 
 cudaError_t launch_gelu(const void* h, int64_t M, int64_t K, int64_t ldh, void* g, int64_t ldg, int sms,
                         cudaStream_t stream) {
+  (void)sms;
+  const LutGeometry geo = lut_geometry<gelu_rows_lut_kernel>(stream);
+  if (geo.cluster == 0) return cudaErrorInvalidConfiguration;
   const int64_t total = M * (K / 8);
-  const int64_t max_blocks = static_cast<int64_t>(sms > 0 ? sms : 148) * 8;
-  const int64_t blocks = std::min<int64_t>(max_blocks, (total + 255) / 256);
-  gelu_rows_kernel<<<static_cast<unsigned>(blocks > 0 ? blocks : 1), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(h), M, K, ldh, static_cast<__nv_bfloat16*>(g), ldg);
-  return cudaGetLastError();
+  const int64_t per_cluster = static_cast<int64_t>(kLutThreads) * geo.cluster;
+  const int64_t clusters = std::max<int64_t>(1, std::min<int64_t>(geo.clusters, (total + per_cluster - 1) / per_cluster));
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(static_cast<unsigned>(clusters * geo.cluster));
+  lc.blockDim = dim3(kLutThreads);
+  lc.dynamicSmemBytes = kLutSmemBytes;
+  lc.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(geo.cluster);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 2;
+  return cudaLaunchKernelEx(&lc, gelu_rows_lut_kernel, static_cast<const __nv_bfloat16*>(h), M, K, ldh,
+                            static_cast<__nv_bfloat16*>(g), ldg, geo.cluster);
 }
 
 cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq,
