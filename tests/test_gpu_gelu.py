@@ -58,7 +58,12 @@ def _act(M, K, seed, scale=4.0):
     return oracle.f32_to_bf16_bits(x)
 
 
-@pytest.mark.parametrize("M,K", [(37, 272), (130, 3072), (17, 4096), (9, 12288), (3, 24592), (2, 40000)])
+# The table kernel at 2, 4, 6 and 8 vectors per thread (K up to 4096, 8192,
+# 12288, 16384; ragged and full), with more rows than row groups in the grid
+# (the persistent loop and its prefetch of the next row: 1500 x 3072,
+# 700 x 12288), and the per-element kernels beyond 16384.
+@pytest.mark.parametrize("M,K", [(37, 272), (130, 3072), (17, 4096), (11, 8192), (7, 6160), (9, 12288),
+                                 (5, 16384), (3, 14352), (1500, 3072), (700, 12288), (3, 24592), (2, 40000)])
 def test_quantize_act_gelu(w8, M, K):
     h = _act(M, K, M + K)
     ht = bf16_bits_to_torch(h, "cuda")

@@ -238,14 +238,18 @@ cudaError_t launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_
 // then the cluster synchronises once.  This happens before the kernel waits
 // for its producer, so it overlaps the tail of the kernel that writes h.
 //
-// Rows: a persistent grid of one 1024-thread CTA per SM; each 256-thread
-// group (four per CTA) quantizes one row at a time, VPL 16-byte vectors per
-// thread held in registers, |GELU(h)| reduced over the group's eight warps
-// through shared memory and a named barrier.
-constexpr int kLutGroups = 4;
-constexpr int kLutThreads = 256 * kLutGroups;
+// Rows: a persistent grid of one CTA per SM (the table leaves room for no
+// second); each 256-thread group of the CTA quantizes one row at a time,
+// VPL 16-byte vectors per thread held in registers, |GELU(h)| reduced over
+// the group's eight warps through shared memory and a named barrier.  While
+// a group looks its row up and encodes it, the loads of its next row are
+// already in flight (a second register copy of the row): a group that only
+// waited for its row and then worked on it left HBM and the shared-memory
+// pipe each less than half busy.
+constexpr int kLutMaxGroups = 4;
+constexpr int kLutThreads = 1024;  // the standalone GELU kernel
 constexpr int kLutTableBytes = 65536 * 2;
-constexpr int kLutSmemBytes = kLutTableBytes + 2 * kLutGroups * 8 * 4;
+constexpr int kLutSmemBytes = kLutTableBytes + 2 * kLutMaxGroups * 8 * 4;
 
 __device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, const uint4& v) {
   asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "r"(v.x), "r"(v.y),
@@ -283,13 +287,14 @@ __device__ __forceinline__ void build_gelu_table(uint16_t* table, int cluster) {
   }
 }
 
-template <int VPL>
-__global__ void __launch_bounds__(kLutThreads, 1)
+template <int VPL, int GROUPS>
+__global__ void __launch_bounds__(256 * GROUPS, 1)
     quantize_rows_gelu_lut_kernel(const __nv_bfloat16* __restrict__ x, int64_t M, int64_t K, int64_t ldx,
                                   int8_t* __restrict__ q, int64_t ldq, float* __restrict__ scale, int cluster) {
+  static_assert(GROUPS >= 1 && GROUPS <= kLutMaxGroups, "row groups per CTA");
   extern __shared__ __align__(16) uint8_t lut_smem[];
   uint16_t* table = reinterpret_cast<uint16_t*>(lut_smem);
-  float* wmax = reinterpret_cast<float*>(lut_smem + kLutTableBytes);  // [2][kLutGroups][8]
+  float* wmax = reinterpret_cast<float*>(lut_smem + kLutTableBytes);  // [2][GROUPS][8]
   const int tid = threadIdx.x;
   build_gelu_table(table, cluster);
   // h is the previous kernel's output: wait for it only now.
@@ -302,16 +307,24 @@ __global__ void __launch_bounds__(kLutThreads, 1)
   const int lane = tid & 31;
   const int warp = t >> 5;
   const int nvec = static_cast<int>(K / 8);
-  int parity = 0;
-  for (int64_t row = static_cast<int64_t>(blockIdx.x) * kLutGroups + grp; row < M;
-       row += static_cast<int64_t>(gridDim.x) * kLutGroups, parity ^= 1) {
-    const uint4* xr = reinterpret_cast<const uint4*>(x + row * ldx);
-    uint4 c[VPL];
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * GROUPS;
+  uint4 next[VPL];
+  auto load_row = [&](int64_t r) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + r * ldx);
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int v = t + 256 * i;
-      c[i] = v < nvec ? __ldg(xr + v) : make_uint4(0u, 0u, 0u, 0u);  // GELU(+0) = +0
+      next[i] = v < nvec ? __ldg(xr + v) : make_uint4(0u, 0u, 0u, 0u);  // GELU(+0) = +0
     }
+  };
+  int64_t row = static_cast<int64_t>(blockIdx.x) * GROUPS + grp;
+  if (row < M) load_row(row);
+  int parity = 0;
+  for (; row < M; row += stride, parity ^= 1) {
+    uint4 c[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) c[i] = next[i];
+    if (row + stride < M) load_row(row + stride);
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
@@ -321,7 +334,7 @@ __global__ void __launch_bounds__(kLutThreads, 1)
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    float* slot = wmax + (parity * kLutGroups + grp) * 8;
+    float* slot = wmax + (parity * GROUPS + grp) * 8;
     if (lane == 0) slot[warp] = amax;
     named_barrier_sync(1 + grp, 256);
 #pragma unroll
@@ -344,7 +357,8 @@ __global__ void __launch_bounds__(kLutThreads, 1)
 }
 
 // bf16 GELU of rows h [M, K] into g by the same table: a persistent grid
-// over the rows' 16-byte vectors, eight lookups per vector.
+// over the rows' 16-byte vectors, four vectors per thread in flight, eight
+// lookups per vector.
 __global__ void __launch_bounds__(kLutThreads, 1)
     gelu_rows_lut_kernel(const __nv_bfloat16* __restrict__ h, int64_t M, int64_t K, int64_t ldh,
                          __nv_bfloat16* __restrict__ g, int64_t ldg, int cluster) {
@@ -354,15 +368,30 @@ __global__ void __launch_bounds__(kLutThreads, 1)
   pdl_wait_prerequisites();
   pdl_launch_dependents();
   cluster_sync_all();
+  constexpr int kUnroll = 4;
   const int64_t vpr = K / 8;  // vectors per row
   const int64_t total = M * vpr;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / vpr;
-    const int64_t v = i - r * vpr;
-    const uint4 x = __ldg(reinterpret_cast<const uint4*>(h + r * ldh) + v);
-    reinterpret_cast<uint4*>(g + r * ldg)[v] =
-        make_uint4(lut_pair(table, x.x), lut_pair(table, x.y), lut_pair(table, x.z), lut_pair(table, x.w));
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < total;
+       base += kUnroll * stride) {
+    uint4 x[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t i = base + u * stride;
+      if (i < total) {
+        const int64_t r = i / vpr;
+        x[u] = __ldg(reinterpret_cast<const uint4*>(h + r * ldh) + (i - r * vpr));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t i = base + u * stride;
+      if (i < total) {
+        const int64_t r = i / vpr;
+        reinterpret_cast<uint4*>(g + r * ldg)[i - r * vpr] = make_uint4(
+            lut_pair(table, x[u].x), lut_pair(table, x[u].y), lut_pair(table, x[u].z), lut_pair(table, x[u].w));
+      }
+    }
   }
 }
 
@@ -373,7 +402,7 @@ struct LutGeometry {
   int clusters = 0;
 };
 
-template <auto kernel>
+template <auto kernel, int kThreads>
 LutGeometry lut_geometry(cudaStream_t stream) {
   constexpr int kMaxDev = 64;
   static std::mutex mu;
@@ -396,7 +425,7 @@ LutGeometry lut_geometry(cudaStream_t stream) {
     for (int c : {8, 4}) {
       cudaLaunchConfig_t lc = {};
       lc.gridDim = dim3(c * (sms / c));
-      lc.blockDim = dim3(kLutThreads);
+      lc.blockDim = dim3(kThreads);
       lc.dynamicSmemBytes = kLutSmemBytes;
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -417,16 +446,27 @@ LutGeometry lut_geometry(cudaStream_t stream) {
   return g;
 }
 
+// Row groups per CTA for VPL vectors per thread: as many as the registers of
+// two copies of the row allow (a CTA of 256 * G threads has 65536 / (256 * G)
+// registers per thread).  At VPL 6 (rows of 12288) three groups would fit
+// with a small spill but measured slower than two: 89.5 against 82.7 us on
+// 9216 x 12288.
+template <int VPL>
+constexpr int lut_groups() {
+  return VPL <= 2 ? 4 : (VPL <= 4 ? 3 : 2);
+}
+
 template <int VPL>
 cudaError_t launch_gelu_lut(const __nv_bfloat16* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq,
                             float* scale, cudaStream_t stream) {
-  const LutGeometry g = lut_geometry<quantize_rows_gelu_lut_kernel<VPL>>(stream);
+  constexpr int G = lut_groups<VPL>();
+  const LutGeometry g = lut_geometry<quantize_rows_gelu_lut_kernel<VPL, G>, 256 * G>(stream);
   if (g.cluster == 0) return cudaErrorInvalidConfiguration;
-  const int64_t rows_per_cluster = static_cast<int64_t>(kLutGroups) * g.cluster;
+  const int64_t rows_per_cluster = static_cast<int64_t>(G) * g.cluster;
   const int64_t clusters = std::min<int64_t>(g.clusters, (M + rows_per_cluster - 1) / rows_per_cluster);
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(static_cast<unsigned>(clusters * g.cluster));
-  lc.blockDim = dim3(kLutThreads);
+  lc.blockDim = dim3(256 * G);
   lc.dynamicSmemBytes = kLutSmemBytes;
   lc.stream = stream;
   cudaLaunchAttribute attr[2];
@@ -438,7 +478,7 @@ cudaError_t launch_gelu_lut(const __nv_bfloat16* x, int64_t M, int64_t K, int64_
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
   lc.numAttrs = 2;
-  return cudaLaunchKernelEx(&lc, quantize_rows_gelu_lut_kernel<VPL>, x, M, K, ldx, q, ldq, scale, g.cluster);
+  return cudaLaunchKernelEx(&lc, quantize_rows_gelu_lut_kernel<VPL, G>, x, M, K, ldx, q, ldq, scale, g.cluster);
 }
 
 }  // namespace
@@ -451,13 +491,13 @@ cudaError_t prepare_quantize_act_gelu(int64_t K, cudaStream_t stream) {
   const int64_t per_thread = (K / 8 + 255) / 256;
   LutGeometry g;
   if (per_thread <= 2) {
-    g = lut_geometry<quantize_rows_gelu_lut_kernel<2>>(stream);
+    g = lut_geometry<quantize_rows_gelu_lut_kernel<2, lut_groups<2>()>, 256 * lut_groups<2>()>(stream);
   } else if (per_thread <= 4) {
-    g = lut_geometry<quantize_rows_gelu_lut_kernel<4>>(stream);
+    g = lut_geometry<quantize_rows_gelu_lut_kernel<4, lut_groups<4>()>, 256 * lut_groups<4>()>(stream);
   } else if (per_thread <= 6) {
-    g = lut_geometry<quantize_rows_gelu_lut_kernel<6>>(stream);
+    g = lut_geometry<quantize_rows_gelu_lut_kernel<6, lut_groups<6>()>, 256 * lut_groups<6>()>(stream);
   } else if (per_thread <= 8) {
-    g = lut_geometry<quantize_rows_gelu_lut_kernel<8>>(stream);
+    g = lut_geometry<quantize_rows_gelu_lut_kernel<8, lut_groups<8>()>, 256 * lut_groups<8>()>(stream);
   } else {
     return cudaSuccess;  // longer rows use the row kernels, which need no setup
   }
@@ -481,7 +521,7 @@ cudaError_t launch_quantize_act_gelu(const void* h, int64_t M, int64_t K, int64_
 cudaError_t launch_gelu(const void* h, int64_t M, int64_t K, int64_t ldh, void* g, int64_t ldg, int sms,
                         cudaStream_t stream) {
   (void)sms;
-  const LutGeometry geo = lut_geometry<gelu_rows_lut_kernel>(stream);
+  const LutGeometry geo = lut_geometry<gelu_rows_lut_kernel, kLutThreads>(stream);
   if (geo.cluster == 0) return cudaErrorInvalidConfiguration;
   const int64_t total = M * (K / 8);
   const int64_t per_cluster = static_cast<int64_t>(kLutThreads) * geo.cluster;
