@@ -109,3 +109,44 @@ def test_chain_layer_with_gelu_input(w8):
     assert np.array_equal(l2["ws_xq"].cpu().numpy(), xq_o)
     assert np.array_equal(torch_bf16_to_bits(l2["out"]), y_o)
     chain.close()
+
+
+_CAPTURE_FIRST = r"""
+import sys
+import numpy as np
+import torch
+sys.path.insert(0, sys.argv[1])
+import oracle
+import w8a8_int8_gemm_b200 as w8
+from tests.test_gpu_gelu import _act
+from tests.util import bf16_bits_to_torch
+h = _act(600, 12288, 21)
+x = bf16_bits_to_torch(h, "cuda")
+q = torch.empty((600, 12288), dtype=torch.int8, device="cuda")
+s = torch.empty((600,), dtype=torch.float32, device="cuda")
+g = torch.cuda.CUDAGraph()
+stream = torch.cuda.Stream()
+with torch.cuda.stream(stream):
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+        w8.w8a8_quantize_act_gelu(x, q, s, stream=stream)
+g.replay()
+torch.cuda.synchronize()
+q_want, s_want = oracle.gelu_quantize_act(h)
+assert np.array_equal(s.cpu().numpy().view(np.uint32), s_want.view(np.uint32)), "scales differ"
+assert np.array_equal(q.cpu().numpy(), q_want), "codes differ"
+print("ok")
+"""
+
+
+def test_quantize_act_gelu_first_call_captured(w8, tmp_path):
+    """A process whose first GELU quantizer call is recorded into a CUDA graph
+    (the table kernel's launch geometry is then the one chosen without the
+    occupancy query, clusters of two) gives the oracle's codes."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    script = tmp_path / "capture_first.py"
+    script.write_text(_CAPTURE_FIRST)
+    out = subprocess.run([sys.executable, str(script), root], capture_output=True, text=True, timeout=600, cwd=root)
+    assert out.returncode == 0 and "ok" in out.stdout, out.stdout[-2000:] + out.stderr[-2000:]
