@@ -299,6 +299,16 @@ W8A8_API w8a8_status w8a8_linear_fp8(const void* x, const uint8_t* wq, const flo
  *   ldh, ldg (multiples of 8 elements), K % 8 == 0.
  * w8a8_linear_gelu: out = GELU(h) W^T + b through w8a8_quantize_act_gelu
  *   and w8a8_gemm; arguments as w8a8_linear.
+ *
+ * Resources.  w8a8_gelu, and w8a8_quantize_act_gelu on rows of up to 16384
+ * elements, look GELU up in a table of all 65536 bf16 inputs that each
+ * launch builds in shared memory (128 KB per CTA, one CTA per SM) with the
+ * same arithmetic; they launch as thread-block clusters of 2 to 8 CTAs,
+ * which share the work of building the table.  The cluster size comes from
+ * an occupancy query made on the first call per device; a first call made
+ * while its stream is being captured uses clusters of 2 instead (same
+ * results).  Longer rows evaluate GELU per element.  A failed cluster
+ * launch returns W8A8_ERR_LAUNCH.
  */
 W8A8_API w8a8_status w8a8_quantize_act_gelu(const void* h, int64_t M, int64_t K, int64_t ldh,
                                             int8_t* xq, int64_t ldxq, float* scale_a, w8a8_stream_t stream);
