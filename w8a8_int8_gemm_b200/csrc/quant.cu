@@ -446,6 +446,33 @@ LutGeometry lut_geometry(cudaStream_t stream) {
   return g;
 }
 
+// Launches a table kernel: `units` work items (rows or vectors), `per_cta`
+// of them per CTA per pass, on at most the clusters that are resident at once
+// (the grid is persistent), as a programmatic dependent of the previous
+// kernel in the stream.  The kernel's last argument is the cluster size.
+template <auto kernel, int kThreads, typename... Args>
+cudaError_t launch_lut(int64_t units, int64_t per_cta, cudaStream_t stream, Args... args) {
+  const LutGeometry geo = lut_geometry<kernel, kThreads>(stream);
+  if (geo.cluster == 0) return cudaErrorInvalidConfiguration;
+  const int64_t per_cluster = per_cta * geo.cluster;
+  const int64_t clusters = std::max<int64_t>(1, std::min<int64_t>(geo.clusters, (units + per_cluster - 1) / per_cluster));
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(static_cast<unsigned>(clusters * geo.cluster));
+  lc.blockDim = dim3(kThreads);
+  lc.dynamicSmemBytes = kLutSmemBytes;
+  lc.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(geo.cluster);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 2;
+  return cudaLaunchKernelEx(&lc, kernel, args..., geo.cluster);
+}
+
 // Row groups per CTA for VPL vectors per thread: as many as the registers of
 // two copies of the row allow (a CTA of 256 * G threads has 65536 / (256 * G)
 // registers per thread).  At VPL 6 (rows of 12288) three groups would fit
@@ -460,25 +487,7 @@ template <int VPL>
 cudaError_t launch_gelu_lut(const __nv_bfloat16* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq,
                             float* scale, cudaStream_t stream) {
   constexpr int G = lut_groups<VPL>();
-  const LutGeometry g = lut_geometry<quantize_rows_gelu_lut_kernel<VPL, G>, 256 * G>(stream);
-  if (g.cluster == 0) return cudaErrorInvalidConfiguration;
-  const int64_t rows_per_cluster = static_cast<int64_t>(G) * g.cluster;
-  const int64_t clusters = std::min<int64_t>(g.clusters, (M + rows_per_cluster - 1) / rows_per_cluster);
-  cudaLaunchConfig_t lc = {};
-  lc.gridDim = dim3(static_cast<unsigned>(clusters * g.cluster));
-  lc.blockDim = dim3(256 * G);
-  lc.dynamicSmemBytes = kLutSmemBytes;
-  lc.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(g.cluster);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  lc.attrs = attr;
-  lc.numAttrs = 2;
-  return cudaLaunchKernelEx(&lc, quantize_rows_gelu_lut_kernel<VPL, G>, x, M, K, ldx, q, ldq, scale, g.cluster);
+  return launch_lut<quantize_rows_gelu_lut_kernel<VPL, G>, 256 * G>(M, G, stream, x, M, K, ldx, q, ldq, scale);
 }
 
 }  // namespace
@@ -520,28 +529,10 @@ cudaError_t launch_quantize_act_gelu(const void* h, int64_t M, int64_t K, int64_
 
 cudaError_t launch_gelu(const void* h, int64_t M, int64_t K, int64_t ldh, void* g, int64_t ldg, int sms,
                         cudaStream_t stream) {
-  (void)sms;
-  const LutGeometry geo = lut_geometry<gelu_rows_lut_kernel, kLutThreads>(stream);
-  if (geo.cluster == 0) return cudaErrorInvalidConfiguration;
-  const int64_t total = M * (K / 8);
-  const int64_t per_cluster = static_cast<int64_t>(kLutThreads) * geo.cluster;
-  const int64_t clusters = std::max<int64_t>(1, std::min<int64_t>(geo.clusters, (total + per_cluster - 1) / per_cluster));
-  cudaLaunchConfig_t lc = {};
-  lc.gridDim = dim3(static_cast<unsigned>(clusters * geo.cluster));
-  lc.blockDim = dim3(kLutThreads);
-  lc.dynamicSmemBytes = kLutSmemBytes;
-  lc.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(geo.cluster);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  lc.attrs = attr;
-  lc.numAttrs = 2;
-  return cudaLaunchKernelEx(&lc, gelu_rows_lut_kernel, static_cast<const __nv_bfloat16*>(h), M, K, ldh,
-                            static_cast<__nv_bfloat16*>(g), ldg, geo.cluster);
+  (void)sms;  // the grid is sized from the cluster occupancy instead
+  return launch_lut<gelu_rows_lut_kernel, kLutThreads>(M * (K / 8), kLutThreads, stream,
+                                                      static_cast<const __nv_bfloat16*>(h), M, K, ldh,
+                                                      static_cast<__nv_bfloat16*>(g), ldg);
 }
 
 cudaError_t launch_quantize_act(const void* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, int64_t ldq,
