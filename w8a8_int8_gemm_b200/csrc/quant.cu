@@ -416,9 +416,12 @@ LutGeometry lut_geometry(cudaStream_t stream) {
   }
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 2) return {};
-  // Clusters of 2 always fit side by side (SMs come in pairs); larger ones
-  // are taken when the occupancy query says that at least as many SMs stay
-  // busy.  The query is not made while the stream is being captured.
+  // Clusters of 2 always fit side by side (SMs come in pairs).  A larger
+  // cluster splits the table's construction over more CTAs; it is taken when
+  // the clusters of that size that are resident at once leave at most
+  // kSpareSms of the SMs idle (per the occupancy query).  The query is not
+  // made while the stream is being captured.
+  constexpr int kSpareSms = 8;
   LutGeometry g{2, sms / 2};
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(stream, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusNone) {
@@ -435,11 +438,14 @@ LutGeometry lut_geometry(cudaStream_t stream) {
       lc.attrs = attr;
       lc.numAttrs = 1;
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, kernel, &lc) == cudaSuccess && n * c >= 2 * (sms / 2) - 8) {
+      if (cudaOccupancyMaxActiveClusters(&n, kernel, &lc) != cudaSuccess) {
+        (void)cudaGetLastError();  // the query's own error: fall back to a smaller cluster
+        continue;
+      }
+      if (n * c >= 2 * (sms / 2) - kSpareSms) {
         g = LutGeometry{c, n};
         break;
       }
-      (void)cudaGetLastError();
     }
     cache[dev] = g;
   }
