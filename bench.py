@@ -964,6 +964,7 @@ def _run_block_on(args, blk, w8, rank, world, local, dev, stream) -> None:
     if args.e2e_steps:
         e2e = block_e2e(args, blk, w8, L, host, dev, stream)
     cpu = block_cpu_baseline(blk) if (world == 1 and not args.no_cpu_baseline) else None
+    block_traffic = ncu_traffic(blk.name, "block")
     cfg = block_config(blk)
     cfg["path"] = "w8a8_chain_launch per step: one CUDA graph of 4 x (quantizer + GEMM)"
     cfg["parallelism"] = f"dp{world} (independent token batches, replicated weights)"
@@ -975,9 +976,10 @@ def _run_block_on(args, blk, w8, rank, world, local, dev, stream) -> None:
         "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded; stands in for Ideogram 4.0 "
         "DiT activations and weights, which are not available)", "config": cfg,
         "roofline": {"bound": "tensor", "achieved": kernel_tops, "peak": int8_peak, "unit": "TOPS",
-                     "frac": kernel_tops / int8_peak, "traffic": None,
+                     "frac": kernel_tops / int8_peak,
+                     "traffic": block_traffic["dram_bytes_per_launch"] if block_traffic else None,
                      "kernel": "gemm_w8a8_kernel over the block's four shapes (sum of their ops / sum of their "
-                               "live launch times)",
+                               "live launch times; traffic: mean DRAM bytes of the four launches)",
                      "ms_per_launch": gemm_total / len(blk.layers),
                      "timing": f"CUDA events around each GEMM launch of the last {R} steps of the timed region",
                      "peak_source": f"{peaks['source']} sustained bf16 {peaks['bf16_tflops_sustained']} TFLOP/s x "
