@@ -33,3 +33,26 @@ def test_warmup_below_three_is_rejected():
            "--steps", "3", "--warmup", "2"]
     out = subprocess.run(cmd, capture_output=True, text=True, timeout=120, cwd=ROOT)
     assert out.returncode != 0
+
+
+def _bench_module():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+@pytest.mark.parametrize("workload,kind", [("mlp_up_1024", "two-kernel"), ("mlp_up_1024", "fp8"),
+                                           ("dit_block_1024", "block")])
+def test_traffic_files_only_count_for_the_sources_they_were_taken_on(monkeypatch, workload, kind):
+    """The committed ncu traffic of a bench line's dominant kernel is reported
+    only while the kernel sources hash to the value recorded with it."""
+    b = _bench_module()
+    with open(os.path.join(ROOT, "profiles", f"dram_{kind}_{workload}.json")) as fh:
+        rec = json.load(fh)
+    assert rec["dram_bytes_per_launch"] > 0
+    monkeypatch.setattr(b, "gemm_source_hash", lambda: rec["gemm_source_hash"])
+    assert b.ncu_traffic(workload, kind)["dram_bytes_per_launch"] == rec["dram_bytes_per_launch"]
+    monkeypatch.setattr(b, "gemm_source_hash", lambda: "0" * 16)
+    assert b.ncu_traffic(workload, kind) is None
