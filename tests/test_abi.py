@@ -123,3 +123,21 @@ def test_host_validation_without_device(w8):
     assert lib.w8a8_gemm_i32_ex(A, A, A, 4, 8, 32, ctypes.byref(cfg), None) == 1
     assert lib.w8a8_select_config(4, 8, 32, None) == 1
     assert lib.w8a8_selftest_wait_timeout(10, None) == 1
+
+
+def test_binding_without_the_library_fails_loudly(tmp_path):
+    """The Python binding has no fallback: a copy of the package without
+    libw8a8.so raises ImportError on import (naming the missing library)."""
+    import os
+    import shutil
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = tmp_path / "w8a8_int8_gemm_b200"
+    pkg.mkdir()
+    shutil.copy(os.path.join(root, "w8a8_int8_gemm_b200", "__init__.py"), pkg / "__init__.py")
+    code = ("import sys; sys.path.insert(0, sys.argv[1])\n"
+            "try:\n    import w8a8_int8_gemm_b200\nexcept ImportError as e:\n    print('ImportError:', e); sys.exit(3)\n"
+            "sys.exit(0)\n")
+    out = subprocess.run([sys.executable, "-c", code, str(tmp_path)], capture_output=True, text=True, timeout=300)
+    assert out.returncode == 3, out.stdout + out.stderr
+    assert "libw8a8.so is missing" in out.stdout
