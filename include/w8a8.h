@@ -356,8 +356,10 @@ typedef struct w8a8_chain_st* w8a8_chain_t;
 
 /* Validates every layer as w8a8_linear does (errors as for w8a8_linear,
  * returned before any CUDA call; count must be 1..4096), then records the
- * chain on the current device.  On success *chain is the new chain; on
- * failure *chain is NULL and nothing stays allocated. */
+ * chain on the current device (layers with input_act = W8A8_ACT_GELU have
+ * their table kernel's cluster geometry set up first, outside the capture).
+ * On success *chain is the new chain; on failure *chain is NULL and nothing
+ * stays allocated. */
 W8A8_API w8a8_status w8a8_chain_create(const w8a8_linear_desc* layers, int32_t count, w8a8_chain_t* chain);
 
 /* Enqueues the whole chain on `stream` (asynchronous, one graph launch).
