@@ -81,14 +81,14 @@ class Oracle:
         lib.oracle_quantize_rows_f32_fp8.argtypes = [p, i64, i64, i64, p, i64, p]
         lib.oracle_gemm_fp8_f64.argtypes = [p, p, i64, i64, i64, p]
         lib.oracle_epilogue_fp8.argtypes = [p, p, p, p, i64, i64, p]
-        lib.oracle_expf.argtypes = [ctypes.c_float]
-        lib.oracle_expf.restype = ctypes.c_float
-        lib.oracle_gelu_f32.argtypes = [ctypes.c_float]
-        lib.oracle_gelu_f32.restype = ctypes.c_float
-        lib.oracle_expf_array.argtypes = [p, i64, p]
-        lib.oracle_expf_array.restype = None
-        lib.oracle_gelu_f32_array.argtypes = [p, i64, p]
-        lib.oracle_gelu_f32_array.restype = None
+        lib.oracle_gelu_f64.argtypes = [ctypes.c_double]
+        lib.oracle_gelu_f64.restype = ctypes.c_double
+        lib.oracle_f64_to_bf16_rne.argtypes = [ctypes.c_double]
+        lib.oracle_f64_to_bf16_rne.restype = ctypes.c_uint16
+        lib.oracle_gelu_f64_array.argtypes = [p, i64, p]
+        lib.oracle_gelu_f64_array.restype = None
+        lib.oracle_f64_to_bf16_array.argtypes = [p, i64, p]
+        lib.oracle_f64_to_bf16_array.restype = None
         lib.oracle_gelu_rows.argtypes = [p, i64, i64, i64, p, i64]
         for fn in ("oracle_quantize_rows_bf16", "oracle_quantize_rows_f32", "oracle_gemm_i64",
                    "oracle_epilogue", "oracle_epilogue_f64", "oracle_linear", "oracle_quantize_rows_bf16_fp8",
@@ -294,18 +294,18 @@ class Oracle:
 
     # --------------------------------------- GELU (producer of X), fused quantizer
 
-    def expf(self, x) -> np.ndarray:
-        """The oracle's own binary32 exp, element-wise."""
-        a = _c(x, np.float32)
+    def gelu_f64(self, x) -> np.ndarray:
+        """GELU (tanh form) in binary64, element-wise, before any bf16 rounding."""
+        a = _c(x, np.float64)
         y = np.empty_like(a)
-        self.lib.oracle_expf_array(_ptr(a), a.size, _ptr(y))
+        self.lib.oracle_gelu_f64_array(_ptr(a), a.size, _ptr(y))
         return y
 
-    def gelu_f32(self, x) -> np.ndarray:
-        """GELU (tanh form) in binary32, element-wise, before any bf16 rounding."""
-        a = _c(x, np.float32)
-        y = np.empty_like(a)
-        self.lib.oracle_gelu_f32_array(_ptr(a), a.size, _ptr(y))
+    def f64_to_bf16_bits(self, x) -> np.ndarray:
+        """float64 -> bf16 bit patterns, rounded once to nearest even."""
+        a = _c(x, np.float64)
+        y = np.empty(a.shape, np.uint16)
+        self.lib.oracle_f64_to_bf16_array(_ptr(a), a.size, _ptr(y))
         return y
 
     def gelu(self, h_bits) -> np.ndarray:
@@ -388,12 +388,12 @@ def epilogue_fp8(acc, scale_a, scale_w, bias_bits=None):
     return get().epilogue_fp8(acc, scale_a, scale_w, bias_bits)
 
 
-def expf(x):
-    return get().expf(x)
+def gelu_f64(x):
+    return get().gelu_f64(x)
 
 
-def gelu_f32(x):
-    return get().gelu_f32(x)
+def f64_to_bf16_bits(x):
+    return get().f64_to_bf16_bits(x)
 
 
 def gelu(h_bits):

@@ -39,18 +39,27 @@
  *   out[m,n]  = bf16_rne( fl32( fl32( fl32(acc)*s_a[m] ) * s_w[n] ) + bias[n] )
  *
  * GELU before a linear layer (the producer of its input, fused with the
- * per-token quantizer on the GPU): the tanh form h / (1 + exp(-2u)),
- * u = sqrt(2/pi) (h + 0.044715 h^3), with this file's own exp (Cody-Waite
- * reduction and a degree-7 Taylor polynomial) and reciprocal (three
- * Newton-Raphson steps), rounded to bf16:
+ * per-token quantizer on the GPU).  The pages name no activation; the one
+ * taken is the tanh form of GELU (Hendrycks & Gimpel, "Gaussian Error
+ * Linear Units"), as DiT MLPs use it, rounded once to bf16 -- what a GELU
+ * kernel stores for the next linear layer:
  *
+ *   gelu(h)   = 0.5 h (1 + tanh(u)),   u = sqrt(2/pi) (h + 0.044715 h^3)
  *   g[r,k]    = bf16_rne( gelu(h[r,k]) ),  then the quantizer above on g
+ *
+ * gelu is evaluated in binary64 through the equal form h / (1 + exp(-2u))
+ * (0.5 (1 + tanh u) = 1 / (1 + exp(-2u))), which, unlike 1 + tanh(u), does
+ * not cancel for negative h, with the C library's exp, and the binary64
+ * value is rounded once to bf16 (no intermediate binary32 rounding).
  *
  * Parity pins (what this file is checked against, other than itself):
  * brute force and closed forms in the CPU test suite -- numpy float32
  * division and rint for the quantizer, numpy int64 matmul and exact
  * integer closed forms for the accumulator, torch's bf16 conversion for
- * the rounding helper, and an fp64 recomputation bounding the epilogue.
+ * the rounding helper, and an fp64 recomputation bounding the epilogue;
+ * for GELU, the correctly rounded bf16 value of the exact function
+ * (60-digit decimal arithmetic) on every bf16 input, exact rational
+ * rounding for the binary64 -> bf16 step, and torch's float64 GELU.
  */
 #include <math.h>
 #include <pthread.h>
@@ -198,80 +207,53 @@ int oracle_epilogue_fp8(const double* acc, const float* scale_a, const float* sc
 
 /* ------------------------------------------------- GELU, the producer of X */
 
-/* exp(x) in binary32, this library's own: Cody-Waite reduction
- * x = k ln2 + r with ln2 split as LN2_HI (low bits zero, so k * LN2_HI is
- * exact for |k| < 2^9) + LN2_LO, k = rint(x * log2 e); the degree-7 Taylor
- * polynomial of exp(r) (|r| <= ln2 / 2 + rounding) by Horner's rule with
- * fused multiply-adds; then one product with 2^k built from its bits.
- * Arguments above 88 give +inf, below -30 give 0 (1 + exp(x) is 1 in
- * binary32 there).  Every step one correctly rounded binary32 operation, in
- * this order, so the GPU reproduces it bit for bit. */
-static const float LOG2E = 1.44269502162933349609375f;    /* fl32(log2 e) */
-static const float LN2_HI = 0.693145751953125f;           /* 0x3F317200 */
-static const float LN2_LO = 1.428606765330187045037746429443359375e-6f;  /* fl32(ln2 - LN2_HI) */
-
-float oracle_expf(float x) {
-    if (x > 88.0f) return INFINITY;
-    if (x < -30.0f) return 0.0f;
-    float k = rintf(x * LOG2E);
-    float r = fmaf(-k, LN2_HI, x);
-    r = fmaf(-k, LN2_LO, r);
-    float p = 1.0f / 5040.0f;
-    p = fmaf(p, r, 1.0f / 720.0f);
-    p = fmaf(p, r, 1.0f / 120.0f);
-    p = fmaf(p, r, 1.0f / 24.0f);
-    p = fmaf(p, r, 1.0f / 6.0f);
-    p = fmaf(p, r, 0.5f);
-    p = fmaf(p, r, 1.0f);
-    p = fmaf(p, r, 1.0f);
-    uint32_t bits = (uint32_t)((int32_t)k + 127) << 23;   /* 2^k, k in [-44, 127] */
-    float scale;
-    memcpy(&scale, &bits, sizeof scale);
-    return p * scale;
+/* Round a binary64 to the nearest bf16, ties to even, in one step (a
+ * binary64 -> binary32 -> bf16 route would round twice).  bf16 has an
+ * 8-bit significand and binary32's exponent range: on [2^E, 2^(E+1)),
+ * E >= -126, its values are the multiples of 2^(E-7); below 2^-126 the
+ * subnormal ones are the multiples of 2^-133.  The quotient by that spacing
+ * is exact (a power-of-two scaling), nearbyint rounds it to an integer with
+ * ties to even, and the product back is a bf16 value (2^128 and beyond is
+ * +-inf). */
+uint16_t oracle_f64_to_bf16_rne(double d) {
+    uint16_t sign = signbit(d) ? 0x8000u : 0x0000u;
+    if (isnan(d)) return (uint16_t)(sign | 0x7FC0u);
+    double a = fabs(d);
+    if (a == 0.0) return sign;
+    if (isinf(a)) return (uint16_t)(sign | 0x7F80u);
+    int e;
+    frexp(a, &e);                  /* a in [2^(e-1), 2^e) */
+    int E = e - 1;
+    if (E < -126) E = -126;        /* the subnormal spacing */
+    double n = nearbyint(ldexp(a, 7 - E));
+    double v = ldexp(n, E - 7);
+    if (v >= 0x1p128) return (uint16_t)(sign | 0x7F80u);
+    float f = (float)v;            /* exact: v is a bf16 value */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(sign | (u >> 16));
 }
 
-/* 1/d for 1 <= d <= 2^120, this library's own: an initial value from the
- * bits of d (the integer 0x7EF311C3 - bits(d), within 12% of 1/d), two
- * Newton-Raphson steps y <- y (2 - d y) (a fused multiply-add and a
- * product each), then one in residual form y <- y + y (1 - d y) (two fused
- * multiply-adds), which lands within an ulp of 1/d and on 1 exactly for
- * d = 1. */
-static float oracle_recip(float d) {
-    uint32_t b;
-    memcpy(&b, &d, sizeof b);
-    uint32_t yb = 0x7EF311C3u - b;
-    float y;
-    memcpy(&y, &yb, sizeof y);
-    y = y * fmaf(-d, y, 2.0f);
-    y = y * fmaf(-d, y, 2.0f);
-    y = fmaf(y, fmaf(-d, y, 1.0f), y);
-    return y;
-}
+/* GELU of h, tanh form, in binary64 (each operation rounded in the order
+ * written; -ffp-contract=off keeps the products and sums separate). */
+static const double GELU_C0 = 0.79788456080286535587989211986876373695;  /* sqrt(2 / pi) */
+static const double GELU_C1 = 0.044715;
 
-/* GELU, tanh form (Hendrycks & Gimpel, "Gaussian Error Linear Units"):
- * 0.5 h (1 + tanh(u)) = h / (1 + exp(-2u)), u = sqrt(2/pi) (h + 0.044715 h^3),
- * each operation rounded to binary32 in the order written, the division
- * taken as h times the reciprocal above; where -2u > 80 (|gelu| < 3e-34)
- * the result is h * 0, a signed zero. */
-static const float GELU_C0 = 0.79788458347320556640625f;  /* fl32(sqrt(2 / pi)) */
-static const float GELU_C1 = 0.044715f;
-
-float oracle_gelu_f32(float h) {
-    float h3 = (h * h) * h;
-    float inner = h + GELU_C1 * h3;
-    float u = GELU_C0 * inner;
-    float x = -2.0f * u;
-    if (x > 80.0f) return h * 0.0f;
-    return h * oracle_recip(1.0f + oracle_expf(x));
+double oracle_gelu_f64(double h) {
+    double h3 = (h * h) * h;
+    double inner = h + GELU_C1 * h3;
+    double u = GELU_C0 * inner;
+    double e = exp(-2.0 * u);      /* +inf for very negative h: h / inf = -0 */
+    return h / (1.0 + e);
 }
 
 /* Element-wise over arrays (for the checks of these two functions). */
-void oracle_expf_array(const float* x, int64_t n, float* y) {
-    for (int64_t i = 0; i < n; ++i) y[i] = oracle_expf(x[i]);
+void oracle_gelu_f64_array(const double* x, int64_t n, double* y) {
+    for (int64_t i = 0; i < n; ++i) y[i] = oracle_gelu_f64(x[i]);
 }
 
-void oracle_gelu_f32_array(const float* x, int64_t n, float* y) {
-    for (int64_t i = 0; i < n; ++i) y[i] = oracle_gelu_f32(x[i]);
+void oracle_f64_to_bf16_array(const double* x, int64_t n, uint16_t* y) {
+    for (int64_t i = 0; i < n; ++i) y[i] = oracle_f64_to_bf16_rne(x[i]);
 }
 
 /* g = bf16_rne(GELU(h)) for bf16 rows h [M, K] (row stride ldh) into g
@@ -279,8 +261,10 @@ void oracle_gelu_f32_array(const float* x, int64_t n, float* y) {
 int oracle_gelu_rows(const uint16_t* h, int64_t M, int64_t K, int64_t ldh, uint16_t* g, int64_t ldg) {
     if (M < 0 || K < 0 || ldh < K || ldg < K) return 1;
     for (int64_t m = 0; m < M; ++m)
-        for (int64_t k = 0; k < K; ++k)
-            g[m * ldg + k] = oracle_f32_to_bf16_rne(oracle_gelu_f32(oracle_bf16_to_f32(h[m * ldh + k])));
+        for (int64_t k = 0; k < K; ++k) {
+            double hv = (double)oracle_bf16_to_f32(h[m * ldh + k]);
+            g[m * ldg + k] = oracle_f64_to_bf16_rne(oracle_gelu_f64(hv));
+        }
     return 0;
 }
 

@@ -51,19 +51,25 @@ MUTANTS = [
      "s += lut[a[m * K + k]] * lut[b[n * K + (K - 1 - k)]];"),
     ("e4m3 epilogue scale_w twice", "d *= scale_a[m];", "d *= scale_w[n];"),
     ("e4m3 epilogue dropped bias", "oracle_f32_to_bf16_rne(d + bn);", "oracle_f32_to_bf16_rne(d);"),
-    # GELU before a linear layer, and its exp
-    ("gelu cubic coefficient 0.04471", "static const float GELU_C1 = 0.044715f;",
-     "static const float GELU_C1 = 0.04471f;"),
-    ("gelu without the cubic term", "float inner = h + GELU_C1 * h3;", "float inner = h;"),
-    ("gelu wrong sign in exp", "float x = -2.0f * u;", "float x = 2.0f * u;"),
-    ("gelu 1 - e", "oracle_recip(1.0f + oracle_expf(x))", "oracle_recip(1.0f - oracle_expf(x))"),
-    ("reciprocal without the residual step", "    y = fmaf(y, fmaf(-d, y, 1.0f), y);\n", ""),
-    ("reciprocal initial value a factor 4 off", "uint32_t yb = 0x7EF311C3u - b;",
-     "uint32_t yb = 0x7DF311C3u - b;"),
-    ("exp without the low part of ln2", "r = fmaf(-k, LN2_LO, r);", ""),
-    ("exp Taylor term r^7 dropped", "float p = 1.0f / 5040.0f;", "float p = 0.0f;"),
-    ("exp scale off by one", "uint32_t bits = (uint32_t)((int32_t)k + 127) << 23;",
-     "uint32_t bits = (uint32_t)((int32_t)k + 128) << 23;"),
+    # GELU before a linear layer (binary64) and the binary64 -> bf16 rounding
+    ("gelu cubic coefficient 0.04471", "static const double GELU_C1 = 0.044715;",
+     "static const double GELU_C1 = 0.04471;"),
+    ("gelu sqrt(2)/pi for sqrt(2/pi)", "static const double GELU_C0 = 0.79788456080286535587989211986876373695;",
+     "static const double GELU_C0 = 0.45015815807855303477759959550337001681;"),
+    ("gelu without the cubic term", "double inner = h + GELU_C1 * h3;", "double inner = h;"),
+    ("gelu wrong sign in exp", "double e = exp(-2.0 * u);", "double e = exp(2.0 * u);"),
+    ("gelu sigmoid(u) for sigmoid(2u)", "double e = exp(-2.0 * u);", "double e = exp(-u);"),
+    ("gelu 1 - e", "return h / (1.0 + e);", "return h / (1.0 - e);"),
+    ("gelu halved twice", "return h / (1.0 + e);", "return 0.5 * h / (1.0 + e);"),
+    ("bf16 from binary64 through binary32 (double rounding)", "double n = nearbyint(ldexp(a, 7 - E));",
+     "double n = nearbyint(ldexp((double)(float)a, 7 - E));"),
+    ("bf16 from binary64 ties away from zero", "double n = nearbyint(ldexp(a, 7 - E));",
+     "double n = round(ldexp(a, 7 - E));"),
+    ("bf16 from binary64 truncated", "double n = nearbyint(ldexp(a, 7 - E));",
+     "double n = trunc(ldexp(a, 7 - E));"),
+    ("bf16 from binary64 subnormal spacing 2^-134", "if (E < -126) E = -126;", "if (E < -127) E = -127;"),
+    ("bf16 from binary64 loses the sign", "uint16_t sign = signbit(d) ? 0x8000u : 0x0000u;",
+     "uint16_t sign = 0x0000u;"),
 ]
 
 
