@@ -103,6 +103,31 @@ def measured_peaks() -> dict:
                 "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def tensor_peak(peaks: dict, region_ms: float, fmt: str = "int8") -> dict:
+    """The dense int8 (or fp8) tensor peak a kernel's roofline fraction is
+    taken against: the measured bf16 cuBLAS figure times the nominal dense
+    int8/bf16 (fp8/bf16) ratio of 2, the burst figure for a kernel timed in a
+    region shorter than a second, the sustained (power-capped) one for a
+    region of a second or more.  detail(achieved) gives the fractions of
+    both and of the 4.5 POPS (PFLOP/s) spec."""
+    sustained = region_ms >= 1000.0
+    burst_peak = peaks["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
+    sus_peak = peaks["bf16_tflops_sustained"] * NOMINAL_INT8_OVER_BF16
+    peak = sus_peak if sustained else burst_peak
+    which = "sustained" if sustained else "burst"
+    src = (f"{peaks['source']} {which} bf16 "
+           f"{peaks['bf16_tflops_sustained'] if sustained else peaks['bf16_tflops']} TFLOP/s x "
+           f"{NOMINAL_INT8_OVER_BF16} (nominal dense {fmt}/bf16 ratio), {which} because the timed region "
+           f"lasted {region_ms:.1f} ms ({'>=' if sustained else '<'} 1 s)")
+
+    def detail(achieved: float) -> dict:
+        return {"peak_kind": which, "peak_source": src, "frac_of_burst_peak": achieved / burst_peak,
+                "frac_of_sustained_peak": achieved / sus_peak, "frac_of_spec_4p5": achieved / SPEC_INT8_POPS,
+                "burst_peak": burst_peak, "sustained_peak": sus_peak}
+
+    return {"peak": peak, "kind": which, "detail": detail}
+
+
 def gemm_source_hash() -> str:
     h = hashlib.sha256()
     for rel in GEMM_SOURCES:
@@ -361,13 +386,16 @@ def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
 
     # The timed region replays CUDA graphs of the step (the host launch cost of
     # the Python binding is not part of the layer); exactly K steps run.  Its
-    # last G steps replay an instrumented graph that brackets every launch of
-    # the dominant kernel (the GEMM) with CUDA events, which gives that
-    # kernel's duration live inside the timed region (those steps launch the
-    # GEMM plainly, without the programmatic overlap the events would break).
+    # last G_inst steps replay an instrumented graph that brackets every
+    # launch of the dominant kernel (the GEMM) with CUDA events, which gives
+    # that kernel's duration live inside the timed region at any step count.
+    # Those steps launch the GEMM plainly, without the programmatic overlap
+    # the events would break, so they are kept to a quarter of the region
+    # (at least one step, at most G).
     G = nsets * max(1, 32 // nsets)
+    G_inst = max(1, min(G, args.steps // 4))
     inst_ev = [(torch.cuda.Event(enable_timing=True, external=True),
-                torch.cuda.Event(enable_timing=True, external=True)) for _ in range(G)]
+                torch.cuda.Event(enable_timing=True, external=True)) for _ in range(G_inst)]
 
     def step_instrumented(i):
         if args.path == "fused":
@@ -380,11 +408,11 @@ def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
             step_gemm(i)
             inst_ev[i][1].record(stream)
 
-    n_graphs = args.steps // G
-    g_main = capture(step, G) if n_graphs > 1 else None
-    g_inst = capture(step_instrumented, G) if n_graphs >= 1 else None
-    g_tail = capture(step, args.steps % G) if args.steps % G else None
-    for g in (g_main, g_inst, g_tail):
+    n_main, n_tail = divmod(args.steps - G_inst, G)
+    g_main = capture(step, G) if n_main else None
+    g_tail = capture(step, n_tail) if n_tail else None
+    g_inst = capture(step_instrumented, G_inst)
+    for g in (g_main, g_tail, g_inst):
         if g is not None:
             g.replay()
     torch.cuda.synchronize(dev)
@@ -397,12 +425,11 @@ def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
     sampler = ClockSampler(local)
     time.sleep(0.3)
     start.record(stream)
-    for _ in range(n_graphs - 1):
+    for _ in range(n_main):
         g_main.replay()
     if g_tail is not None:
         g_tail.replay()
-    if g_inst is not None:
-        g_inst.replay()
+    g_inst.replay()
     end.record(stream)
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
@@ -412,7 +439,7 @@ def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
     code = w8.w8a8_read_device_error()
     if code != 0:
         raise SystemExit(f"a kernel wait timed out in the timed region (site {code})")
-    live_kernel_ms = (statistics.fmean(a.elapsed_time(b) for a, b in inst_ev) if g_inst is not None else None)
+    live_kernel_ms = statistics.fmean(a.elapsed_time(b) for a, b in inst_ev)
 
     ms_step = elapsed_ms / args.steps
     ops = 2.0 * M * N * K
@@ -437,17 +464,26 @@ def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
         return a_ev.elapsed_time(b_ev) / (reps * G)
 
     peaks = measured_peaks()
-    # The GEMM is timed inside a seconds-long loop under the board's power
-    # cap: its peak is the sustained bf16 figure times the nominal ratio.
-    int8_peak = peaks["bf16_tflops_sustained"] * NOMINAL_INT8_OVER_BF16
-    int8_peak_burst = peaks["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
     quant_bytes = 3 * M * K + 4 * M
-    kernel_fn = step_fused if args.path == "fused" else step_gemm
-    kernel_ms = live_kernel_ms if live_kernel_ms is not None else graph_ms(kernel_fn, max(3, 300 // G))
+    kernel_ms = live_kernel_ms
     kernel_tops = ops / (kernel_ms * 1e-3) / 1e12
+    roof_peak = tensor_peak(peaks, elapsed_ms, "fp8" if fp8 else "int8")
     side = {}
     if rank == 0 and not args.no_context:
-        side["quant_ms"] = graph_ms(step_quant, max(3, 300 // G))
+        # the quantizer on its own rotation of inputs and outputs (> 3x L2 of its
+        # bytes; the layer's buffer sets hold too few quantizer bytes for that)
+        nq = max(2, int(np.ceil(3 * L2_BYTES / quant_bytes)))
+        qsets = [(sets[0]["x"] if i == 0 else torch.roll(sets[0]["x"], shifts=i, dims=0).contiguous(),
+                  torch.empty((M, K), dtype=code_dtype, device=dev),
+                  torch.empty((M,), dtype=torch.float32, device=dev)) for i in range(nq)]
+
+        def step_quant_rotating(i):
+            x, xq, sa = qsets[i % nq]
+            quantize_act(x, xq=xq, scale_a=sa, stream=stream)
+
+        side["quant_ms"] = time_graph(step_quant_rotating, stream, dev, nq * max(1, 24 // nq), max(3, 300 // G))
+        side["quant_rotation_mb"] = round(nq * quant_bytes / 2 ** 20, 1)
+        del qsets
         side["gemm_ms"] = graph_ms(step_gemm, max(3, 300 // G))
         side["linear_ms"] = graph_ms(step_linear, max(3, 300 // G))
         if not fp8:
@@ -475,13 +511,16 @@ def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
         e2e = run_e2e(w8, wl, x_host, sets[0]["wq"], sw, bias, dev, stream, args) if args.e2e_steps else None
         ctx = context_baselines(wl, d, sets, sw, bias, dev, args, graph_ms) if not args.no_context else None
         cpu = cpu_baseline(wl, fp8=fp8) if (world == 1 and not args.no_cpu_baseline) else None
+        table = (per_config_table(w8, dev, stream, peaks, cpu=world == 1 and not args.no_cpu_baseline)
+                 if (not args.no_per_config and not fp8) else None)
         cfg = wl_config(wl)
         cfg["format"] = "fp8 (OCP E4M3 codes, fp32 accumulation)" if fp8 else "int8 (int32 accumulation)"
         cfg["path"] = ("one fused kernel per step (w8a8_linear_fused)" if args.path == "fused"
                        else f"{linear.__name__} per step: quantizer kernel, then the GEMM kernel as its "
                             "programmatic dependent")
-        cfg["timing"] = (f"CUDA graphs of {G} steps replayed (the last {G} steps instrumented); events around "
-                         "the whole timed region")
+        cfg["timing"] = (f"CUDA graphs of {G} steps replayed, the last {G_inst} steps an instrumented graph "
+                         f"(events around each GEMM); events around the whole timed region "
+                         f"({elapsed_ms:.1f} ms)")
         cfg["parallelism"] = f"dp{world} (independent token batches, replicated weight)"
         cfg["gemm_config"] = w8.w8a8_select_config(M, N, K)
         cfg["buffer_sets"] = nsets
@@ -495,19 +534,16 @@ def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
             "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3" if fp8 else "int8",
             "data": "synthetic (seeded; stands in for Ideogram 4.0 "
             "DiT activations and weights, which are not available)", "config": cfg,
-            "roofline": {"bound": "tensor", "achieved": kernel_tops, "peak": int8_peak, "unit": unit,
-                         "frac": kernel_tops / int8_peak,
-                         "traffic": traffic["dram_bytes_per_launch"] if traffic else None,
-                         "kernel": kname, "ms_per_launch": kernel_ms,
-                         "timing": f"CUDA events around each of the last {G} launches of this kernel inside "
-                                   "the timed region (on the launching stream)",
-                         "peak_source": f"{peaks['source']} sustained bf16 {peaks['bf16_tflops_sustained']} "
-                                        f"TFLOP/s x {NOMINAL_INT8_OVER_BF16} (nominal dense "
-                                        f"{'fp8' if fp8 else 'int8'}/bf16 ratio)",
-                         "frac_of_burst_peak": kernel_tops / int8_peak_burst},
+            "roofline": dict({"bound": "tensor", "achieved": kernel_tops, "peak": roof_peak["peak"],
+                              "unit": unit, "frac": kernel_tops / roof_peak["peak"],
+                              "traffic": traffic["dram_bytes_per_launch"] if traffic else None,
+                              "kernel": kname, "ms_per_launch": kernel_ms,
+                              "timing": f"CUDA events around each of the last {G_inst} launches of this kernel "
+                                        "inside the timed region (on the launching stream)"},
+                             **roof_peak["detail"](kernel_tops)),
             ("pct_of_spec_fp8_4p5_pflops" if fp8 else "pct_of_spec_int8_4p5_pops"): 100 * kernel_tops / SPEC_INT8_POPS,
             "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
-            "cpu_baseline": cpu, "context": ctx,
+            "cpu_baseline": cpu, "context": ctx, "per_config": table,
         }
         if side:
             result["components"] = {
@@ -516,6 +552,7 @@ def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
             if "quant_ms" in side:
                 qg = quant_bytes / (side["quant_ms"] * 1e-3) / 1e9
                 result["components"]["quantizer"] = {"ms": side["quant_ms"], "gbs": qg,
+                                                     "rotation_mb": side["quant_rotation_mb"],
                                                      "frac_of_measured_hbm": qg / peaks["hbm_gbs"],
                                                      "frac_of_8tbs": qg / 8000.0, "bytes": quant_bytes}
                 if "copy_ms" in side:
@@ -657,6 +694,160 @@ def context_baselines(wl, d, sets, sw, bias, dev, args, graph_ms) -> dict:
         out[fn.__name__] = {"ms": ms, "tops": 2.0 * M * N * K / (ms * 1e-3) / 1e12}
     del w_sets, w_bf16, acc32
     return out
+
+
+# ------------------------------------------------------ per-config table
+
+# Every linear-layer configuration of the DiT workloads (QKV at 768px; the
+# 1024px MLP up- and long-K down-projection; the four layers of the full-block
+# sweep at batch 2, 1024px + 512 text tokens), each measured on its own in the
+# same run as the headline line.
+PER_CONFIG = ["qkv_768", "mlp_up_1024", "mlp_down_1024", "sweep_qkv", "sweep_out", "sweep_up", "sweep_down"]
+
+
+def time_graph(fn, stream, dev, n: int, reps: int) -> float | None:
+    """Mean ms per call of fn(i): a CUDA graph of n back-to-back calls
+    (i = 0..n-1), replayed reps times between CUDA events on `stream`."""
+    g = torch.cuda.CUDAGraph()
+    try:
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+            for i in range(n):
+                fn(i)
+    except RuntimeError as exc:
+        print(f"[bench] could not capture {getattr(fn, '__name__', fn)}: {exc}", file=sys.stderr)
+        torch.cuda.synchronize(dev)
+        return None
+    g.replay()
+    a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a_ev.record(stream)
+    for _ in range(reps):
+        g.replay()
+    b_ev.record(stream)
+    torch.cuda.synchronize(dev)
+    return a_ev.elapsed_time(b_ev) / (reps * n)
+
+
+def measure_config(w8, wl, dev, stream, peaks: dict, cpu: bool) -> dict:
+    """One configuration, every entry point timed the same way: CUDA graphs
+    of back-to-back calls cycling through buffer sets whose combined size is
+    more than 3x L2, so operands come from HBM.  The seeded inputs of the
+    workload; int8-given workloads (long-K MLP down) have no quantizer."""
+    M, N, K = wl.M, wl.N, wl.K
+    d = workloads.make(wl)
+    linear_kind = wl.kind == "linear"
+    bias = torch.from_numpy(d["bias"].view(np.int16)).view(torch.bfloat16).to(dev)
+    if linear_kind:
+        wq0, sw = w8.w8a8_quantize_weight(torch.from_numpy(d["w"]).to(dev))
+        x0 = torch.from_numpy(d["x"].view(np.int16)).view(torch.bfloat16).to(dev)
+        w_bf = torch.from_numpy(d["w"]).to(dev).to(torch.bfloat16)
+        set_bytes = M * K * 2 + M * K + N * K + N * K * 2 + M * N * 2 + 4 * M
+    else:
+        wq0 = torch.from_numpy(d["wq"]).to(dev)
+        sw = torch.from_numpy(d["scale_w"]).to(dev)
+        xq0 = torch.from_numpy(d["xq"]).to(dev)
+        sa0 = torch.from_numpy(d["scale_a"]).to(dev)
+        # the bf16 context runs on the dequantized operands
+        x0 = (xq0.float() * sa0[:, None]).to(torch.bfloat16)
+        w_bf = (wq0.float() * sw[:, None]).to(torch.bfloat16)
+        set_bytes = M * K * 2 + M * K + N * K + N * K * 2 + M * N * 2 + 4 * M
+    nsets = max(2, int(np.ceil(3 * L2_BYTES / set_bytes)))
+    sets = []
+    for i in range(nsets):
+        s = {"x": x0 if i == 0 else torch.roll(x0, shifts=i, dims=0).contiguous(),
+             "wq": wq0 if i == 0 else wq0.clone(), "w_bf": w_bf if i == 0 else w_bf.clone(),
+             "out": torch.empty((M, N), dtype=torch.bfloat16, device=dev)}
+        if linear_kind:
+            s["xq"] = torch.empty((M, K), dtype=torch.int8, device=dev)
+            s["sa"] = torch.empty((M,), dtype=torch.float32, device=dev)
+            w8.w8a8_quantize_act(s["x"], xq=s["xq"], scale_a=s["sa"], stream=stream)
+        else:
+            s["xq"] = xq0 if i == 0 else torch.roll(xq0, shifts=i, dims=0).contiguous()
+            s["sa"] = sa0 if i == 0 else torch.roll(sa0, shifts=i, dims=0).contiguous()
+        sets.append(s)
+    torch.cuda.synchronize(dev)
+
+    def gemm(i):
+        s = sets[i % nsets]
+        w8.w8a8_gemm(s["xq"], s["wq"], s["sa"], sw, bias, out=s["out"], stream=stream)
+
+    def linear(i):
+        s = sets[i % nsets]
+        w8.w8a8_linear(s["x"], s["wq"], sw, bias, out=s["out"], ws_xq=s["xq"], ws_scale_a=s["sa"], stream=stream)
+
+    # the quantizer alone moves far fewer bytes than the layer: its own
+    # rotation of inputs and outputs, more than 3x L2 in all
+    qbytes = 3 * M * K + 4 * M
+    nq = max(2, int(np.ceil(3 * L2_BYTES / qbytes))) if linear_kind else 0
+    qsets = [(x0 if i == 0 else torch.roll(x0, shifts=i, dims=0).contiguous(),
+              torch.empty((M, K), dtype=torch.int8, device=dev), torch.empty((M,), dtype=torch.float32, device=dev))
+             for i in range(nq)]
+
+    def quant(i):
+        x, xq, sa = qsets[i % nq]
+        w8.w8a8_quantize_act(x, xq=xq, scale_a=sa, stream=stream)
+
+    def bf16_matmul(i):
+        s = sets[i % nsets]
+        torch.addmm(bias, s["x"], s["w_bf"].t(), out=s["out"])
+
+    def dequant_to_bf16_path(i):
+        # the production "INT8" forward the paper replaces: quantize, dequantize to bf16, bf16 GEMM
+        s = sets[i % nsets]
+        xf = s["x"].float()
+        sa = xf.abs().amax(dim=1, keepdim=True) / 127.0
+        xq = torch.clamp(torch.round(xf / torch.where(sa > 0, sa, torch.ones_like(sa))), -127, 127)
+        wd = (s["wq"].float() * sw[:, None]).to(torch.bfloat16)
+        torch.addmm(bias, (xq * sa).to(torch.bfloat16), wd.t(), out=s["out"])
+
+    n = nsets * max(1, 12 // nsets)
+    ops = 2.0 * M * N * K
+    res = {"workload": wl.name, "M": M, "N": N, "K": K, "buffer_sets": nsets,
+           "footprint_mb": round(nsets * set_bytes / 2 ** 20, 1)}
+    for fn in (bf16_matmul, dequant_to_bf16_path):   # library handles are created outside graph capture
+        fn(0)
+    torch.cuda.synchronize(dev)
+    gms = time_graph(gemm, stream, dev, n, 5)
+    res["gemm_us"] = 1e3 * gms
+    res["gemm_tops"] = ops / (gms * 1e-3) / 1e12
+    res["gemm_pct_of_spec_4p5"] = 100 * res["gemm_tops"] / SPEC_INT8_POPS
+    res["gemm_frac_of_burst_peak"] = res["gemm_tops"] / (peaks["bf16_tflops"] * NOMINAL_INT8_OVER_BF16)
+    res["gemm_config"] = w8.w8a8_select_config(M, N, K)
+    if linear_kind:
+        lms = time_graph(linear, stream, dev, n, 5)
+        qms = time_graph(quant, stream, dev, nq * max(1, 24 // nq), 5)
+        res["quant_rotation_mb"] = round(nq * qbytes / 2 ** 20, 1)
+        res["linear_us"] = 1e3 * lms
+        res["linear_tops"] = ops / (lms * 1e-3) / 1e12
+        res["linear_pct_of_spec_4p5"] = 100 * res["linear_tops"] / SPEC_INT8_POPS
+        res["quant_us"] = 1e3 * qms
+        res["quant_gbs"] = qbytes / (qms * 1e-3) / 1e9
+        res["quant_frac_of_measured_hbm"] = res["quant_gbs"] / peaks["hbm_gbs"]
+        res["quant_frac_of_8tbs"] = res["quant_gbs"] / 8000.0
+    for fn in (bf16_matmul, dequant_to_bf16_path):
+        ms = time_graph(fn, stream, dev, n, 3)
+        res[fn.__name__ + "_us"] = None if ms is None else 1e3 * ms
+    if cpu:
+        work = OracleWork(wl, pool_rows=256)
+        rows, cols = size_sample(work, 1.5)
+        dt = work.sample(rows, cols)
+        res["oracle"] = {"tops": 2.0 * rows * cols * K / dt / 1e12, "cores": work.threads,
+                         "sample": f"{rows} tokens x {cols} channels, {dt:.2f} s",
+                         "full_layer_s_extrapolated": dt * (M * N) / (rows * cols)}
+    del sets, qsets, x0, w_bf, wq0
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    return res
+
+
+def per_config_table(w8, dev, stream, peaks: dict, cpu: bool) -> dict:
+    sampler = ClockSampler(dev.index)
+    rows = [measure_config(w8, workloads.WORKLOADS[name], dev, stream, peaks, cpu) for name in PER_CONFIG]
+    return {"note": "after the timed region, each configuration on its own: CUDA graphs of back-to-back calls "
+                    "over rotating buffer sets (> 3x L2); GEMM = w8a8_gemm (quantized operands given), linear = "
+                    "w8a8_linear (quantizer + GEMM), quant = w8a8_quantize_act; bf16_matmul = torch.addmm; "
+                    "dequant_to_bf16_path = quantize, dequantize to bf16, bf16 GEMM (the path the paper "
+                    "replaces); oracle = the CPU oracle on a row x column sample of the whole layer",
+            "clocks": sampler.stop(), "configs": rows}
 
 
 # ------------------------------------------------------- DiT block chain
@@ -901,7 +1092,7 @@ def _run_block_on(args, blk, w8, rank, world, local, dev, stream) -> None:
     kernel_tops = blk.ops / (gemm_total * 1e-3) / 1e12
 
     peaks = measured_peaks()
-    int8_peak = peaks["bf16_tflops_sustained"] * NOMINAL_INT8_OVER_BF16
+    roof_peak = tensor_peak(peaks, elapsed_ms)
     if rank != 0:
         chain.close()
         return
@@ -975,15 +1166,14 @@ def _run_block_on(args, blk, w8, rank, world, local, dev, stream) -> None:
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded; stands in for Ideogram 4.0 "
         "DiT activations and weights, which are not available)", "config": cfg,
-        "roofline": {"bound": "tensor", "achieved": kernel_tops, "peak": int8_peak, "unit": "TOPS",
-                     "frac": kernel_tops / int8_peak,
-                     "traffic": block_traffic["dram_bytes_per_launch"] if block_traffic else None,
-                     "kernel": "gemm_w8a8_kernel over the block's four shapes (sum of their ops / sum of their "
-                               "live launch times; traffic: mean DRAM bytes of the four launches)",
-                     "ms_per_launch": gemm_total / len(blk.layers),
-                     "timing": f"CUDA events around each GEMM launch of the last {R} steps of the timed region",
-                     "peak_source": f"{peaks['source']} sustained bf16 {peaks['bf16_tflops_sustained']} TFLOP/s x "
-                                    f"{NOMINAL_INT8_OVER_BF16} (nominal dense int8/bf16 ratio)"},
+        "roofline": dict({"bound": "tensor", "achieved": kernel_tops, "peak": roof_peak["peak"], "unit": "TOPS",
+                          "frac": kernel_tops / roof_peak["peak"],
+                          "traffic": block_traffic["dram_bytes_per_launch"] if block_traffic else None,
+                          "kernel": "gemm_w8a8_kernel over the block's four shapes (sum of their ops / sum of "
+                                    "their live launch times; traffic: mean DRAM bytes of the four launches)",
+                          "ms_per_launch": gemm_total / len(blk.layers),
+                          "timing": f"CUDA events around each GEMM launch of the last {R} steps of the timed "
+                                    "region"}, **roof_peak["detail"](kernel_tops)),
         "components": comps, "e2e": e2e, "gpu_launches": 2 * len(blk.layers) * steps, "clocks": clocks,
         "cpu_baseline": cpu, "context": ctx,
     }
@@ -1007,6 +1197,8 @@ def main(argv=None) -> int:
                     help="int8 W8A8 (default) or its FP8 (E4M3) variant")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-context", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the table of every DiT configuration measured after the headline")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -284,13 +284,15 @@ W8A8_API w8a8_status w8a8_linear_fp8(const void* x, const uint8_t* wq, const flo
  * up- and down-projections).  Unfused, a GELU kernel writes bf16 G =
  * GELU(H) to HBM and the quantizer reads it back; fused, one pass reads H and
  * writes the codes, saving a write and a read of G.  GELU is the tanh form
- * (Hendrycks & Gimpel, "Gaussian Error Linear Units") written as
- *   gelu(h) = h / (1 + exp(-2u)),  u = sqrt(2/pi) * (h + 0.044715 h^3),
- * each step one binary32 operation in that order, exp the library's own
- * (Cody-Waite reduction by ln 2 and a degree-7 Taylor polynomial, fused
- * multiply-adds; +inf above 88, 0 below -30), rounded to bf16: exactly what
- * w8a8_gelu stores.  The pages name no activation; this is the library's
- * definition.
+ * (Hendrycks & Gimpel, "Gaussian Error Linear Units"),
+ *   gelu(h) = 0.5 h (1 + tanh(u)),  u = sqrt(2/pi) * (h + 0.044715 h^3),
+ * evaluated in binary64 as h / (1 + exp(-2u)) (the same function, without
+ * the cancellation of 1 + tanh(u) for negative h) and rounded once to bf16:
+ * exactly what w8a8_gelu stores.  That is the correctly rounded bf16 value
+ * of gelu(h) for every bf16 input except the 256 of magnitude below 2^-125
+ * with an odd last bit, where gelu(h) = h/2 + O(h^2) lies within 1e-40
+ * (relative) of a bf16 midpoint: there the result is bf16_rne(h/2).  The
+ * pages name no activation; this is the library's definition.
  *
  * w8a8_quantize_act_gelu: codes and scales of bf16_rne(gelu(h)); arguments
  *   as w8a8_quantize_act (h in place of x).  Bit-identical to w8a8_gelu
@@ -303,10 +305,11 @@ W8A8_API w8a8_status w8a8_linear_fp8(const void* x, const uint8_t* wq, const flo
  * Resources.  w8a8_gelu, and w8a8_quantize_act_gelu on rows of up to 16384
  * elements, look GELU up in a table of all 65536 bf16 inputs that each
  * launch builds in shared memory (128 KB per CTA, one CTA per SM) with the
- * same arithmetic; they launch as thread-block clusters of 2 to 8 CTAs,
- * which share the work of building the table.  The cluster size comes from
- * an occupancy query made on the first call per device; a first call made
- * while its stream is being captured uses clusters of 2 instead (same
+ * same binary64 arithmetic; they launch as thread-block clusters of 2 to 8
+ * CTAs, which share the work of building the table.  The cluster size comes from
+ * an occupancy query, made once per device by the first call whose stream
+ * is not being captured and kept for the process; calls recorded in a stream
+ * capture before that use clusters of 2 and do not keep them (same
  * results).  Longer rows evaluate GELU per element.  A failed cluster
  * launch returns W8A8_ERR_LAUNCH.
  */

@@ -31,7 +31,7 @@ def test_exports_match_header(w8):
 
 def test_status_strings(w8):
     assert w8.w8a8_status_string(0) == "ok"
-    for s in range(1, 7):
+    for s in range(1, 8):
         assert w8.w8a8_status_string(s) not in ("ok", "unknown status")
     assert w8.w8a8_status_string(99) == "unknown status"
     assert w8.w8a8_abi_version() == 101
@@ -101,6 +101,19 @@ def test_host_validation_without_device(w8):
     assert lib.w8a8_gelu(A, 0, 16, 16, A, 16, None) == 0                    # empty
     assert lib.w8a8_linear_gelu(A, A, A, None, A, A, A, 4, 12, 32, None) == 1
     assert lib.w8a8_linear_gelu(A, A, A, None, A, A + 1, A, 4, 8, 32, None) == 2
+    # the no-allocation layer: w8a8_linear's checks, in its order, before the
+    # device check, which comes before the scratch capacity (so an invalid call
+    # that is also too large is an argument error, not a capacity error)
+    assert lib.w8a8_linear_noalloc(A, A, A, None, A, 4, 12, 32, None) == 1         # N % 8
+    assert lib.w8a8_linear_noalloc(A, A, A, None, A, 9000, 8, 24, None) == 1       # K % 16
+    assert lib.w8a8_linear_noalloc(None, A, A, None, A, 4, 8, 32, None) == 1       # no x
+    assert lib.w8a8_linear_noalloc(A, A, A, None, None, 4, 8, 32, None) == 1       # no out
+    assert lib.w8a8_linear_noalloc(A + 8, A, A, None, A, 4, 8, 32, None) == 2      # misaligned x
+    assert lib.w8a8_linear_noalloc(A, A, A, A + 2, A, 4, 8, 32, None) == 2         # misaligned bias
+    assert lib.w8a8_linear_noalloc(A, A, A, None, A, 0, 8, 32, None) == 0          # empty
+    big = lib.w8a8_linear_noalloc(A, A, A, None, A, 1 << 16, 8, 4096, None)        # valid, 256 MiB of codes
+    import torch
+    assert big == 7 if torch.cuda.is_available() else big in (3, 6), big  # no device here: not a capacity error
     # chains of linear layers: every layer is validated before any CUDA call
     h = ctypes.c_void_p(None)
     assert lib.w8a8_chain_create(None, 1, ctypes.byref(h)) == 1

@@ -15,15 +15,14 @@ input for it, so whole chains are compared for equality, output by output
   this method); MLP up 3072->12288 on the attention output's result; MLP
   down 12288->3072 on GELU of MLP up's result, the GELU fused into MLP
   down's quantizer (the norm is not part of this method).  Weights quantized on the GPU are
-  checked against the oracle's; the chain is checked on sampled rows (rows
-  are independent through every layer)."""
+  checked against the oracle's; the chain is checked on every row."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import workloads
-from tests.util import bf16_bits_to_torch, sample_rows, torch_bf16_to_bits
+from tests.util import bf16_bits_to_torch, row_chunks, torch_bf16_to_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -85,43 +84,44 @@ def test_small_chain_all_rows(w8):
 
 
 def test_dit_block_1024_batch2(w8):
-    """The four linears of one DiT block at M = 9216 as one graph."""
+    """The four linears of one DiT block at M = 9216 as one graph, every
+    row: the oracle runs the block layer by layer on chunks of rows (rows are
+    independent through every layer), each layer fed the oracle's own output
+    of the layer before (GELU'd for MLP down)."""
     blk = workloads.BLOCKS["dit_block_1024"]
     M = blk.M
     d = blk.inputs()
     dev = torch.device("cuda")
     src_t = {"x": bf16_bits_to_torch(d["x"], dev), "a": bf16_bits_to_torch(d["a"], dev)}
-    src_o = {"x": d["x"], "a": d["a"]}
-    rows = sample_rows(M, 40, 31)
-    L, ref = {}, {}
+    L, wo = {}, {}
     for l in blk.layers:
         w = d["w_" + l.name]
         wq, sw = w8.w8a8_quantize_weight(torch.from_numpy(w).to(dev))
         torch.cuda.synchronize()
         wq_o, sw_o = oracle.quantize_weight(w)
         assert np.array_equal(wq.cpu().numpy(), wq_o) and np.array_equal(sw.cpu().numpy(), sw_o)
-        b = d["bias_" + l.name]
+        wo[l.name] = (wq_o, sw_o)
         act = w8.ACT_GELU if l.act == "gelu" else w8.ACT_NONE
-        L[l.name] = w8.linear_layer(src_t[l.source], wq, sw, bf16_bits_to_torch(b, dev), input_act=act)
+        L[l.name] = w8.linear_layer(src_t[l.source], wq, sw, bf16_bits_to_torch(d["bias_" + l.name], dev),
+                                    input_act=act)
         src_t[l.name] = L[l.name]["out"]
-        # block inputs are sliced to the sampled rows; earlier layers' oracle
-        # outputs already hold only those rows
-        x_rows = src_o[l.source][rows] if l.source in ("x", "a") else src_o[l.source]
-        if l.act == "gelu":
-            x_rows = oracle.gelu(x_rows)
-        ref[l.name] = _oracle_layer(x_rows, wq_o, sw_o, b)
-        src_o[l.name] = ref[l.name][0]
     chain = w8.w8a8_chain_create([L[l.name] for l in blk.layers])
     chain.launch()
     torch.cuda.synchronize()
     assert w8.w8a8_read_device_error() == 0
-    for l in blk.layers:
-        out_o, xq_o, sa_o = ref[l.name]
-        assert np.array_equal(L[l.name]["ws_xq"].cpu().numpy()[rows], xq_o), l.name
-        assert np.array_equal(L[l.name]["ws_scale_a"].cpu().numpy()[rows], sa_o), l.name
-        assert np.array_equal(torch_bf16_to_bits(L[l.name]["out"])[rows], out_o), l.name
-        assert not torch.isnan(L[l.name]["out"]).any()
+    got = {l.name: (torch_bf16_to_bits(L[l.name]["out"]), L[l.name]["ws_xq"].cpu().numpy(),
+                    L[l.name]["ws_scale_a"].cpu().numpy()) for l in blk.layers}
     chain.close()
+    for rows in row_chunks(M):
+        src_o = {"x": d["x"][rows], "a": d["a"][rows]}
+        for l in blk.layers:
+            x_rows = oracle.gelu(src_o[l.source]) if l.act == "gelu" else src_o[l.source]
+            out_o, xq_o, sa_o = _oracle_layer(x_rows, *wo[l.name], d["bias_" + l.name])
+            src_o[l.name] = out_o
+            out_g, xq_g, sa_g = got[l.name]
+            assert np.array_equal(xq_g[rows], xq_o), (l.name, rows)
+            assert np.array_equal(sa_g[rows].view(np.uint32), sa_o.view(np.uint32)), (l.name, rows)
+            assert np.array_equal(out_g[rows], out_o), (l.name, rows)
 
 
 def test_chain_errors(w8):

@@ -14,7 +14,7 @@ import torch
 
 import oracle
 import workloads
-from tests.util import bf16_bits_to_torch, bf16_ulp_diff, is_nan_bits, sample_rows, torch_bf16_to_bits
+from tests.util import bf16_bits_to_torch, bf16_ulp_diff, is_nan_bits, row_chunks, torch_bf16_to_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -136,16 +136,31 @@ def test_i32_identity_and_extremes(w8):
     assert acc[0, 0] == big and acc[0, 1] == -big and acc[1, 0] == -big and acc[1, 1] == big
 
 
-def test_i32_long_k_workload_sampled(w8):
-    """MLP down-projection 4096 x 3072 x 12288 with the all-+-127 rows, on
-    sampled rows (the whole launch runs; the oracle checks 64+ rows)."""
+def test_long_k_workload_every_row(w8):
+    """MLP down-projection 4096 x 3072 x 12288 with the all-+-127 rows, in
+    the launch configuration the benchmark selects: the int32 accumulators
+    of w8a8_gemm_i32 and the bf16 outputs of w8a8_gemm (dequantization +
+    bias epilogue) against the oracle on every row (its exact GEMM in row
+    chunks); the closed form K * 127^2 on the extreme rows."""
     wl = workloads.WORKLOADS["mlp_down_1024"]
     d = workloads.make(wl)
-    acc = _i32(w8, d["xq"], d["wq"])
-    rows = sample_rows(wl.M, 48, 17)
-    want = oracle.gemm_i64(d["xq"][rows], d["wq"])
-    assert np.array_equal(acc[rows], want)
-    assert acc[0, 0] == wl.K * 127 * 127 and acc[1, 0] == -wl.K * 127 * 127
+    dev = torch.device("cuda")
+    xq, wq = torch.from_numpy(d["xq"]).to(dev), torch.from_numpy(d["wq"]).to(dev)
+    acc = w8.w8a8_gemm_i32(xq, wq)
+    out = w8.w8a8_gemm(xq, wq, torch.from_numpy(d["scale_a"]).to(dev), torch.from_numpy(d["scale_w"]).to(dev),
+                       bf16_bits_to_torch(d["bias"], dev))
+    torch.cuda.synchronize()
+    assert w8.w8a8_read_device_error() == 0
+    acc = acc.cpu().numpy()
+    got = torch_bf16_to_bits(out)
+    assert not is_nan_bits(got).any()
+    big = wl.K * 127 * 127
+    assert acc[0, 0] == big and acc[1, 0] == -big and acc[0, 1] == -big and acc[1, 1] == big
+    for rows in row_chunks(wl.M):
+        want = oracle.gemm_i64(d["xq"][rows], d["wq"])
+        assert np.array_equal(acc[rows], want), f"accumulators differ in rows {rows}"
+        bf = oracle.epilogue(want, d["scale_a"][rows], d["scale_w"], d["bias"])
+        assert bf16_ulp_diff(got[rows], bf).max() <= 1, f"outputs differ in rows {rows}"
 
 
 def test_i32_matches_torch_int_mm(w8):
@@ -192,22 +207,6 @@ def test_bf16_epilogue(w8, M, N, K, bias):
 def test_bf16_epilogue_configs(w8, cfg):
     got, want = _bf16_gemm_case(w8, 300, 776, 656, cfg["block_n"] + cfg["stages"], True, cfg)
     assert bf16_ulp_diff(got, want).max() <= 1
-
-
-def test_bf16_long_k_workload_sampled(w8):
-    """The fused GEMM on the 4096 x 3072 x 12288 workload, sampled rows."""
-    wl = workloads.WORKLOADS["mlp_down_1024"]
-    d = workloads.make(wl)
-    dev = torch.device("cuda")
-    out = w8.w8a8_gemm(torch.from_numpy(d["xq"]).to(dev), torch.from_numpy(d["wq"]).to(dev),
-                       torch.from_numpy(d["scale_a"]).to(dev), torch.from_numpy(d["scale_w"]).to(dev),
-                       bf16_bits_to_torch(d["bias"], dev))
-    torch.cuda.synchronize()
-    got = torch_bf16_to_bits(out)
-    assert not is_nan_bits(got).any()
-    rows = sample_rows(wl.M, 48, 23)
-    want = oracle.epilogue(oracle.gemm_i64(d["xq"][rows], d["wq"]), d["scale_a"][rows], d["scale_w"], d["bias"])
-    assert bf16_ulp_diff(got[rows], want).max() <= 1
 
 
 def test_empty_problem(w8):

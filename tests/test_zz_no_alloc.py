@@ -8,8 +8,10 @@ the library.  These tests call it through the C ABI and check that its
 output equals w8a8_linear's (within the 1-ulp bf16 tolerance of the other
 tests; in practice bit-identical, the kernels are the same) on two calls in
 a row -- the second call finds the first call's leftovers in the shared
-array -- and that a problem larger than the array is refused without
-touching the output.  This file is collected last on purpose."""
+array --, at the size the header advertises (also against the CPU oracle)
+and at the largest size that fits, and that a problem larger than the
+array, by 4 bytes or by far, is refused without touching the output.  This
+file is collected last on purpose."""
 import numpy as np
 import pytest
 import torch
@@ -57,6 +59,52 @@ def test_noalloc_matches_linear_on_two_calls_in_a_row():
         assert bf16_ulp_diff(got, torch_bf16_to_bits(ref)).max() <= 1
 
 
+def test_noalloc_at_the_advertised_size_matches_the_oracle():
+    """9216 tokens x K = 3072 (the size the header gives as fitting) against
+    w8a8_linear and against the CPU oracle on every row."""
+    import oracle
+    import w8a8_int8_gemm_b200 as w8
+    from tests.util import bf16_bits_to_torch
+    import workloads
+    dev = torch.device("cuda")
+    M, N, K = 9216, 1032, 3072
+    x_bits = workloads.gen_activations(M, K, seed=91)
+    w = workloads.gen_weight(N, K, 92)
+    b_bits = workloads.gen_bias(N, 93)
+    x = bf16_bits_to_torch(x_bits, dev)
+    bias = bf16_bits_to_torch(b_bits, dev)
+    wq, sw = w8.w8a8_quantize_weight(torch.from_numpy(w).to(dev))
+    ref = w8.w8a8_linear(x, wq, sw, bias)
+    out = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=dev)
+    assert _noalloc_raw(w8, x, wq, sw, bias, out) == 0
+    torch.cuda.synchronize()
+    assert w8.w8a8_read_device_error() == 0
+    got = torch_bf16_to_bits(out)
+    assert np.array_equal(got, torch_bf16_to_bits(ref))
+    wq_o, sw_o = oracle.quantize_weight(w)
+    want, *_ = oracle.linear(x_bits, wq_o, sw_o, b_bits)
+    assert bf16_ulp_diff(got, want).max() <= 1
+
+
+# The scratch holds M*K codes rounded up to 256 bytes, then 4*M bytes of
+# scales, in 32 MiB: at K = 864, 38656 tokens leave 1024 bytes free and
+# 38657 need 4 bytes more than there are.
+EDGE_K, EDGE_M_FITS = 864, 38656
+
+
+def test_noalloc_at_the_edge_of_its_scratch():
+    import w8a8_int8_gemm_b200 as w8
+    dev = torch.device("cuda")
+    M, N, K = EDGE_M_FITS, 136, EDGE_K
+    assert (M * K + 255) // 256 * 256 + 4 * M == (32 << 20) - 1024
+    x, wq, sw, bias = _inputs(M, N, K, 5, dev)
+    ref = w8.w8a8_linear(x, wq, sw, bias)
+    out = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=dev)
+    assert _noalloc_raw(w8, x, wq, sw, bias, out) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+
+
 def test_noalloc_refuses_problems_beyond_its_scratch():
     import w8a8_int8_gemm_b200 as w8
     dev = torch.device("cuda")
@@ -70,3 +118,12 @@ def test_noalloc_refuses_problems_beyond_its_scratch():
     torch.cuda.synchronize()
     assert bool((out == 3.0).all()), "a refused call must not write the output"
     assert "scratch" in w8.w8a8_status_string(SCRATCH_LIMIT)
+    # 4 bytes beyond the scratch
+    M, K = EDGE_M_FITS + 1, EDGE_K
+    assert (M * K + 255) // 256 * 256 + 4 * M == (32 << 20) + 4
+    x = torch.zeros((M, K), dtype=torch.bfloat16, device=dev)
+    wq = torch.zeros((N, K), dtype=torch.int8, device=dev)
+    out = torch.full((M, N), 3.0, dtype=torch.bfloat16, device=dev)
+    assert _noalloc_raw(w8, x, wq, sw, bias, out) == SCRATCH_LIMIT
+    torch.cuda.synchronize()
+    assert bool((out == 3.0).all())

@@ -37,3 +37,10 @@ def sample_rows(M: int, n: int, seed: int) -> np.ndarray:
     extra = rng.choice(M, size=min(n, M), replace=False)
     rows = np.unique(np.array([r for r in fixed if 0 <= r < M] + list(extra), dtype=np.int64))
     return rows
+
+
+def row_chunks(M: int, chunk: int = 2048):
+    """Row slices covering 0..M in pieces of `chunk` rows: full-size oracle
+    comparisons run piece by piece, so the oracle's int64 accumulators stay a
+    few hundred MB whatever M * N is."""
+    return [slice(r, min(M, r + chunk)) for r in range(0, M, chunk)]

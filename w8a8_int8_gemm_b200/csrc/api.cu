@@ -185,6 +185,29 @@ w8a8_status quantize_common(bool act, const void* x, int64_t M, int64_t K, int64
 }
 
 }  // namespace
+
+// The checks w8a8_linear makes on its shapes and on its caller-owned inputs
+// and output before any CUDA call (workspaces aside): shape, non-null
+// pointers, 16-byte alignment.  W8A8_OK for an empty problem too.
+w8a8_status check_linear_io(const void* x, const int8_t* wq, const float* scale_w, const void* bias,
+                            const void* out, int64_t M, int64_t N, int64_t K) {
+  w8a8_status st = check_gemm_shape(M, N, K);
+  if (st != W8A8_OK) return st;
+  if (M == 0 || N == 0) return W8A8_OK;
+  if (x == nullptr || wq == nullptr || scale_w == nullptr || out == nullptr) return W8A8_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(wq) || !aligned16(scale_w) || !aligned16(bias) || !aligned16(out)) {
+    return W8A8_ERR_ALIGNMENT;
+  }
+  return W8A8_OK;
+}
+
+// W8A8_OK if the current device is supported (sm_100), from the cached
+// device properties.
+w8a8_status check_current_device() {
+  DeviceInfo dev;
+  return current_device(&dev);
+}
+
 }  // namespace w8a8
 
 using namespace w8a8;

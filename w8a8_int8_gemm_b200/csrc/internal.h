@@ -5,6 +5,8 @@
 
 #include <cstdint>
 
+#include "../../include/w8a8.h"
+
 namespace w8a8 {
 
 // Tile configuration of the GEMM kernel (see w8a8_gemm_config in w8a8.h).
@@ -79,6 +81,12 @@ int gemm_max_stages(int block_m, int block_n);
 cudaError_t launch_gemm(const GemmArgs& args, const GemmConfig& cfg, cudaStream_t stream);
 
 cudaError_t launch_selftest_wait(uint64_t timeout_ns, cudaStream_t stream);
+
+// Argument checks of w8a8_linear on its shapes, inputs and output (not the
+// workspaces), made before any CUDA call; and the current device's support.
+w8a8_status check_linear_io(const void* x, const int8_t* wq, const float* scale_w, const void* bias,
+                            const void* out, int64_t M, int64_t N, int64_t K);
+w8a8_status check_current_device();
 
 // Synchronizes the current device and reads (optionally clears) the device
 // error word written by timed-out waits.

@@ -21,6 +21,7 @@
 #include <mutex>
 
 #include "../../include/w8a8.h"
+#include "internal.h"
 
 namespace w8a8 {
 namespace {
@@ -59,13 +60,14 @@ cudaError_t scratch_address(uint8_t** out) {
 extern "C" w8a8_status w8a8_linear_noalloc(const void* x, const int8_t* wq, const float* scale_w, const void* bias,
                                            void* out, int64_t M, int64_t N, int64_t K, w8a8_stream_t stream) {
   using namespace w8a8;
-  // Shapes are validated by w8a8_linear; here only the scratch capacity.
-  if (M < 0 || K < 0) return W8A8_ERR_INVALID_ARG;
-  if (M == 0 || N == 0) return w8a8_linear(x, wq, scale_w, bias, out, nullptr, nullptr, M, N, K, stream);
+  // The same checks as w8a8_linear, in the same order, before any CUDA
+  // call; then the device; only then the scratch capacity and its address.
+  w8a8_status st = check_linear_io(x, wq, scale_w, bias, out, M, N, K);
+  if (st != W8A8_OK) return st;
+  if (M == 0 || N == 0) return W8A8_OK;
+  if ((st = check_current_device()) != W8A8_OK) return st;
   const int64_t code_bytes = (M * K + 255) / 256 * 256;  // scales start 256-byte aligned
-  if (M > kScratchBytes || K > kScratchBytes || code_bytes + 4 * M > kScratchBytes) {
-    return W8A8_ERR_SCRATCH_LIMIT;
-  }
+  if (code_bytes + 4 * M > kScratchBytes) return W8A8_ERR_SCRATCH_LIMIT;
   uint8_t* base = nullptr;
   if (scratch_address(&base) != cudaSuccess) return W8A8_ERR_CUDA;
   int8_t* xq = reinterpret_cast<int8_t*>(base);

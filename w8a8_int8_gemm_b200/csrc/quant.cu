@@ -37,7 +37,9 @@
 // division for every pair of bf16 values |x| <= amax and on 10^9 planted
 // fp32 elements.  Rows whose scale is below 2^-100 (where the remainder can
 // underflow), or whose reciprocal is not finite, take IEEE division
-// (__fdiv_rn) for every element.
+// (__fdiv_rn) for every element, and so do all fp32 rows (weights): they are
+// quantized once at load time, where the division costs nothing that
+// matters, and the shortcut's check covers bf16 inputs exhaustively only.
 //
 // FP8 variant (OCP E4M3 codes; B200's native FP8 path, the comparison
 // baseline of the same paper): the same scheme with 448, the largest finite
@@ -229,10 +231,10 @@ cudaError_t launch_quantize(const T* x, int64_t M, int64_t K, int64_t ldx, int8_
 // GELU fused into the per-token quantizer, by table.  GELU's input is bf16,
 // so it takes one of 65536 values, and what the quantizer consumes,
 // bf16_rne(GELU(h)), is a function of the 16 input bits alone.  The kernel
-// evaluates that function for every bit pattern with the same packed
-// arithmetic the other kernels apply element by element (gelu_bf16x8), into
-// a 128 KB table in shared memory, and then replaces the ~31 instructions of
-// GELU per element by one shared-memory load.  The table is built by a
+// evaluates that function for every bit pattern with the binary64
+// arithmetic the long-row kernels apply element by element (gelu_bf16x8),
+// into a 128 KB table in shared memory, and then replaces GELU per element
+// (a binary64 exp and division) by one shared-memory load.  The table is built by a
 // cluster of CTAs: each computes 65536 / cluster entries and stores them into
 // the shared memory of every CTA of the cluster (distributed shared memory),
 // then the cluster synchronises once.  This happens before the kernel waits
@@ -271,7 +273,7 @@ __device__ __forceinline__ uint32_t lut_pair(const uint16_t* table, uint32_t w) 
 
 // The table of bf16_rne(GELU(h)) for every bf16 bit pattern h, built by a
 // cluster: this CTA computes 65536 / cluster consecutive entries (8 per
-// packed evaluation) and stores each 16-byte run into the table of every CTA
+// call of gelu_bf16x8) and stores each 16-byte run into the table of every CTA
 // of the cluster.  The caller synchronises the cluster before any lookup.
 __device__ __forceinline__ void build_gelu_table(uint16_t* table, int cluster) {
   const uint32_t rank = cluster_ctarank();

@@ -53,74 +53,33 @@ __device__ __forceinline__ uint64_t add(uint64_t a, uint64_t b) {
 __device__ __forceinline__ uint64_t neg(uint64_t a) { return a ^ 0x8000000080000000ull; }
 }  // namespace f2
 
-// GELU of two binary32 values, as the library defines it: the tanh form
-// (Hendrycks & Gimpel) h / (1 + exp(-2u)), u = sqrt(2/pi) (h + 0.044715 h^3),
-// each step one correctly rounded binary32 operation in this order (the
-// pair's lanes computed together by packed instructions):
-//   * exp(x), x = -2u, the library's own: Cody-Waite reduction x = k ln2 + r
-//     (ln2 split so that k * ln2_hi is exact), the degree-7 Taylor polynomial
-//     of exp(r) by Horner's rule with fused multiply-adds, one product with
-//     2^k built from its bits; 0 below -30 (it is evaluated at -30 there and
-//     discarded);
-//   * the division as h times the library's reciprocal of d = 1 + exp(x): an
-//     initial value from the bits of d (0x7EF311C3 - bits(d)), two
-//     Newton-Raphson steps y (2 - d y), one residual step y + y (1 - d y);
-//   * where x > 80 the result is h * 0, a signed zero.
-// No approximate hardware function is used, so the result is reproducible
-// bit for bit off the GPU.
-__device__ __forceinline__ void gelu_f32x2(float& a, float& b) {
-  const uint64_t h = f2::pack(a, b);
-  const uint64_t h3 = f2::mul(f2::mul(h, h), h);
-  const uint64_t inner = f2::add(h, f2::mul(f2::splat(0x1.6e4e26p-5f), h3));  // 0.044715
-  const uint64_t u = f2::mul(f2::splat(0x1.988454p-1f), inner);                // sqrt(2/pi)
-  float x0, x1;
-  f2::unpack(f2::mul(f2::splat(-2.0f), u), x0, x1);
-  const uint64_t xc = f2::pack(fminf(fmaxf(x0, -30.0f), 80.0f), fminf(fmaxf(x1, -30.0f), 80.0f));
-  float t0, t1;
-  f2::unpack(f2::mul(xc, f2::splat(0x1.715476p+0f)), t0, t1);  // log2 e
-  const float k0 = rintf(t0), k1 = rintf(t1);
-  const uint64_t nk = f2::pack(-k0, -k1);
-  uint64_t r = f2::fma(nk, f2::splat(0x1.62e4p-1f), xc);    // ln2, high part
-  r = f2::fma(nk, f2::splat(0x1.7f7d1cp-20f), r);           // ln2, low part
-  uint64_t p = f2::splat(0x1.a01a02p-13f);                  // 1/5040
-  p = f2::fma(p, r, f2::splat(0x1.6c16c2p-10f));            // 1/720
-  p = f2::fma(p, r, f2::splat(0x1.111112p-7f));             // 1/120
-  p = f2::fma(p, r, f2::splat(0x1.555556p-5f));             // 1/24
-  p = f2::fma(p, r, f2::splat(0x1.555556p-3f));             // 1/6
-  p = f2::fma(p, r, f2::splat(0.5f));
-  p = f2::fma(p, r, f2::splat(1.0f));
-  p = f2::fma(p, r, f2::splat(1.0f));
-  float e0, e1;
-  f2::unpack(f2::mul(p, f2::pack(__int_as_float((static_cast<int>(k0) + 127) << 23),
-                                 __int_as_float((static_cast<int>(k1) + 127) << 23))),
-             e0, e1);
-  const uint64_t d = f2::add(f2::splat(1.0f), f2::pack(x0 < -30.0f ? 0.0f : e0, x1 < -30.0f ? 0.0f : e1));
-  float d0, d1;
-  f2::unpack(d, d0, d1);
-  uint64_t y = f2::pack(__uint_as_float(0x7EF311C3u - __float_as_uint(d0)),
-                        __uint_as_float(0x7EF311C3u - __float_as_uint(d1)));
-  const uint64_t nd = f2::neg(d);
-  y = f2::mul(y, f2::fma(nd, y, f2::splat(2.0f)));
-  y = f2::mul(y, f2::fma(nd, y, f2::splat(2.0f)));
-  y = f2::fma(y, f2::fma(nd, y, f2::splat(1.0f)), y);
-  float g0, g1;
-  f2::unpack(f2::mul(h, y), g0, g1);
-  a = x0 > 80.0f ? __fmul_rn(a, 0.0f) : g0;
-  b = x1 > 80.0f ? __fmul_rn(b, 0.0f) : g1;
+// GELU of one bf16 value (bit pattern in the low 16 bits of hb), as the
+// library defines it: the tanh form (Hendrycks & Gimpel, "Gaussian Error
+// Linear Units"), 0.5 h (1 + tanh(u)) with u = sqrt(2/pi) (h + 0.044715 h^3),
+// rounded once to bf16 (nearest, ties to even).  It is evaluated in binary64
+// through the equal form h / (1 + exp(-2u)), which does not cancel for
+// negative h: every product and sum rounded on its own in the order
+// written (no contraction into fused multiply-adds), CUDA's binary64 exp,
+// an IEEE division, then one rounding from binary64 to bf16.  The binary64
+// value is within far less than 2^-40 (relative) of the exact function, so
+// the result is its correctly rounded bf16 value except where that lies
+// nearer a rounding boundary than this error.
+__device__ __forceinline__ uint32_t gelu_bf16_bits(uint32_t hb) {
+  const double h = static_cast<double>(__uint_as_float(hb << 16));
+  const double h3 = __dmul_rn(__dmul_rn(h, h), h);
+  const double inner = __dadd_rn(h, __dmul_rn(0.044715, h3));
+  const double u = __dmul_rn(0.79788456080286535587989211986876373695, inner);  // sqrt(2/pi)
+  const double e = exp(__dmul_rn(-2.0, u));  // +inf for very negative h: h / inf = -0
+  return __bfloat16_as_ushort(__double2bfloat16(__ddiv_rn(h, __dadd_rn(1.0, e))));
 }
 
 // Eight bf16 -> bf16_rne(GELU) of each (what a GELU kernel would store).
-__device__ __forceinline__ uint4 gelu_bf16x8(const uint4& v) {
+// One out-of-line copy: the row kernels apply it to every vector of a row.
+static __device__ __noinline__ uint4 gelu_bf16x8(uint4 v) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t o[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float lo = __uint_as_float(w[i] << 16);
-    float hi = __uint_as_float(w[i] & 0xFFFF0000u);
-    gelu_f32x2(lo, hi);
-    const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-    o[i] = *reinterpret_cast<const uint32_t*>(&b);
-  }
+#pragma unroll 1
+  for (int i = 0; i < 4; ++i) o[i] = gelu_bf16_bits(w[i] & 0xFFFFu) | (gelu_bf16_bits(w[i] >> 16) << 16);
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
@@ -249,10 +208,13 @@ __device__ __forceinline__ uint64_t quotient2(uint64_t x, uint64_t r2, uint64_t 
 // rounds the quotient to an integer n (ties to even; 1.5*2^23 is even) and
 // the low byte of its bit pattern is n's two's-complement int8 code; |x/s|
 // <= 127.0001 keeps n inside [-127, 127] without a clamp.
+// fp32 rows (weights, quantized once at load time) always divide: the
+// shortcut's equality with the division was checked exhaustively on bf16
+// inputs only.
 template <typename T>
 __device__ __forceinline__ void quantize_vec(const uint4& v, const RowScale& rs, int8_t* dst) {
   constexpr int E = Vec<T>::kElems;
-  if (rs.fast) {
+  if (sizeof(T) == 2 && rs.fast) {
     float f[E];
     Vec<T>::unpack(v, f);
     const uint64_t r2 = f2::splat(rs.r), neg_s2 = f2::splat(-rs.s), round2 = f2::splat(12582912.0f);
@@ -280,7 +242,7 @@ __device__ __forceinline__ void quantize_vec_e4m3(const uint4& v, const RowScale
   float f[E];
   Vec<T>::unpack(v, f);
   float d[E];
-  if (rs.fast) {
+  if (sizeof(T) == 2 && rs.fast) {  // fp32 rows (weights) divide, as for int8 codes
     const uint64_t r2 = f2::splat(rs.r), neg_s2 = f2::splat(-rs.s);
 #pragma unroll
     for (int i = 0; i < E; i += 2) {
