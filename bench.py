@@ -484,10 +484,12 @@ def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
         side["quant_ms"] = time_graph(step_quant_rotating, stream, dev, nq * max(1, 24 // nq), max(3, 300 // G))
         side["quant_rotation_mb"] = round(nq * quant_bytes / 2 ** 20, 1)
         del qsets
-        side["gemm_ms"] = graph_ms(step_gemm, max(3, 300 // G))
-        side["linear_ms"] = graph_ms(step_linear, max(3, 300 // G))
-        if not fp8:
-            side["fused_ms"] = graph_ms(step_fused, max(3, 300 // G))
+        if fp8 or args.no_per_config:
+            # int8 runs time every entry point of every configuration in per_config
+            side["gemm_ms"] = graph_ms(step_gemm, max(3, 300 // G))
+            side["linear_ms"] = graph_ms(step_linear, max(3, 300 // G))
+            if not fp8:
+                side["fused_ms"] = graph_ms(step_fused, max(3, 300 // G))
         # the floor for the quantizer's byte count: a plain device copy moving
         # the same bytes (half read, half written), same harness, same rotation
         # (its own rotation, combined footprint > 3x L2, so that it is HBM traffic)
@@ -509,10 +511,14 @@ def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
     result = None
     if rank == 0:
         e2e = run_e2e(w8, wl, x_host, sets[0]["wq"], sw, bias, dev, stream, args) if args.e2e_steps else None
-        ctx = context_baselines(wl, d, sets, sw, bias, dev, args, graph_ms) if not args.no_context else None
+        with_table = not args.no_per_config and not fp8
+        ctx = (context_baselines(wl, d, sets, sw, bias, dev, args, graph_ms)
+               if not args.no_context and not with_table else
+               {"see": "per_config (bf16_matmul, dequant_to_bf16_path, torch_int_mm_no_epilogue)"} if with_table
+               else None)
         cpu = cpu_baseline(wl, fp8=fp8) if (world == 1 and not args.no_cpu_baseline) else None
         table = (per_config_table(w8, dev, stream, peaks, cpu=world == 1 and not args.no_cpu_baseline)
-                 if (not args.no_per_config and not fp8) else None)
+                 if with_table else None)
         cfg = wl_config(wl)
         cfg["format"] = "fp8 (OCP E4M3 codes, fp32 accumulation)" if fp8 else "int8 (int32 accumulation)"
         cfg["path"] = ("one fused kernel per step (w8a8_linear_fused)" if args.path == "fused"
@@ -547,7 +553,9 @@ def _run_native_on(args, wl, w8, rank, world, local, dev, stream) -> None:
         }
         if side:
             result["components"] = {
-                "note": "after the timed region: graphs of back-to-back calls of one entry point",
+                "note": "after the timed region: graphs of back-to-back calls of one entry point"
+                        + ("" if not with_table else "; the GEMM, linear and fused entry points of every "
+                           "configuration, this one included, are in per_config"),
             }
             if "quant_ms" in side:
                 qg = quant_bytes / (side["quant_ms"] * 1e-3) / 1e9
@@ -790,6 +798,20 @@ def measure_config(w8, wl, dev, stream, peaks: dict, cpu: bool) -> dict:
         s = sets[i % nsets]
         torch.addmm(bias, s["x"], s["w_bf"].t(), out=s["out"])
 
+    sync = [torch.zeros((w8.w8a8_linear_sync_words(M),), dtype=torch.int32, device=dev) for _ in range(nsets)]
+
+    def fused(i):
+        s = sets[i % nsets]
+        w8.w8a8_linear_fused(s["x"], s["wq"], sw, bias, out=s["out"], ws_xq=s["xq"], ws_scale_a=s["sa"],
+                             ws_sync=sync[i % nsets], stream=stream)
+
+    acc32 = [torch.empty((M, N), dtype=torch.int32, device=dev) for _ in range(2)]
+
+    def torch_int_mm_no_epilogue(i):
+        # the library int8 GEMM (cuBLAS through torch) with int32 output, no dequantization
+        s = sets[i % nsets]
+        torch._int_mm(s["xq"], s["wq"].t(), out=acc32[i % 2])
+
     def dequant_to_bf16_path(i):
         # the production "INT8" forward the paper replaces: quantize, dequantize to bf16, bf16 GEMM
         s = sets[i % nsets]
@@ -803,9 +825,6 @@ def measure_config(w8, wl, dev, stream, peaks: dict, cpu: bool) -> dict:
     ops = 2.0 * M * N * K
     res = {"workload": wl.name, "M": M, "N": N, "K": K, "buffer_sets": nsets,
            "footprint_mb": round(nsets * set_bytes / 2 ** 20, 1)}
-    for fn in (bf16_matmul, dequant_to_bf16_path):   # library handles are created outside graph capture
-        fn(0)
-    torch.cuda.synchronize(dev)
     gms = time_graph(gemm, stream, dev, n, 5)
     res["gemm_us"] = 1e3 * gms
     res["gemm_tops"] = ops / (gms * 1e-3) / 1e12
@@ -813,6 +832,8 @@ def measure_config(w8, wl, dev, stream, peaks: dict, cpu: bool) -> dict:
     res["gemm_frac_of_burst_peak"] = res["gemm_tops"] / (peaks["bf16_tflops"] * NOMINAL_INT8_OVER_BF16)
     res["gemm_config"] = w8.w8a8_select_config(M, N, K)
     if linear_kind:
+        fms = time_graph(fused, stream, dev, n, 5)
+        res["fused_us"] = None if fms is None else 1e3 * fms
         lms = time_graph(linear, stream, dev, n, 5)
         qms = time_graph(quant, stream, dev, nq * max(1, 24 // nq), 5)
         res["quant_rotation_mb"] = round(nq * qbytes / 2 ** 20, 1)
@@ -823,7 +844,13 @@ def measure_config(w8, wl, dev, stream, peaks: dict, cpu: bool) -> dict:
         res["quant_gbs"] = qbytes / (qms * 1e-3) / 1e9
         res["quant_frac_of_measured_hbm"] = res["quant_gbs"] / peaks["hbm_gbs"]
         res["quant_frac_of_8tbs"] = res["quant_gbs"] / 8000.0
-    for fn in (bf16_matmul, dequant_to_bf16_path):
+    for fn in (bf16_matmul, dequant_to_bf16_path, torch_int_mm_no_epilogue):
+        try:
+            fn(0)
+            torch.cuda.synchronize(dev)
+        except (RuntimeError, TypeError) as exc:  # not supported by this torch / device
+            res[fn.__name__ + "_us"] = {"unavailable": str(exc).splitlines()[0][:160]}
+            continue
         ms = time_graph(fn, stream, dev, n, 3)
         res[fn.__name__ + "_us"] = None if ms is None else 1e3 * ms
     if cpu:
@@ -833,7 +860,7 @@ def measure_config(w8, wl, dev, stream, peaks: dict, cpu: bool) -> dict:
         res["oracle"] = {"tops": 2.0 * rows * cols * K / dt / 1e12, "cores": work.threads,
                          "sample": f"{rows} tokens x {cols} channels, {dt:.2f} s",
                          "full_layer_s_extrapolated": dt * (M * N) / (rows * cols)}
-    del sets, qsets, x0, w_bf, wq0
+    del sets, qsets, x0, w_bf, wq0, acc32, sync
     torch.cuda.synchronize(dev)
     torch.cuda.empty_cache()
     return res
@@ -843,10 +870,12 @@ def per_config_table(w8, dev, stream, peaks: dict, cpu: bool) -> dict:
     sampler = ClockSampler(dev.index)
     rows = [measure_config(w8, workloads.WORKLOADS[name], dev, stream, peaks, cpu) for name in PER_CONFIG]
     return {"note": "after the timed region, each configuration on its own: CUDA graphs of back-to-back calls "
-                    "over rotating buffer sets (> 3x L2); GEMM = w8a8_gemm (quantized operands given), linear = "
-                    "w8a8_linear (quantizer + GEMM), quant = w8a8_quantize_act; bf16_matmul = torch.addmm; "
-                    "dequant_to_bf16_path = quantize, dequantize to bf16, bf16 GEMM (the path the paper "
-                    "replaces); oracle = the CPU oracle on a row x column sample of the whole layer",
+                    "over rotating buffer sets (> 3x L2); gemm = w8a8_gemm (quantized operands given), linear = "
+                    "w8a8_linear (quantizer + GEMM), fused = w8a8_linear_fused (one kernel), quant = "
+                    "w8a8_quantize_act (its own rotation); bf16_matmul = torch.addmm; dequant_to_bf16_path = "
+                    "quantize, dequantize to bf16, bf16 GEMM (the path the paper replaces); "
+                    "torch_int_mm_no_epilogue = the library int8 GEMM, int32 out; oracle = the CPU oracle on a "
+                    "row x column sample of the whole layer",
             "clocks": sampler.stop(), "configs": rows}
 
 
@@ -1109,15 +1138,33 @@ def _run_block_on(args, blk, w8, rank, world, local, dev, stream) -> None:
         torch.cuda.synchronize(dev)
         return a_ev.elapsed_time(b_ev) / (reps * G)
 
-    comps = {"note": "after the timed region, one layer at a time: graphs of back-to-back calls (operands "
-                     "larger than L2 except where noted)"}
+    comps = {"note": "after the timed region, one layer at a time: graphs of back-to-back calls; each quantizer "
+                     "on its own rotation of inputs larger than 3x L2 in all; the linear layers' operands and "
+                     "outputs are larger than L2"}
+    def quantize_rotating_ms(t, K):
+        """The layer's quantizer on its own rotation of inputs and outputs, more
+        than 3x L2 in all (one input of 85 MB would stay in L2)."""
+        nq = max(1, int(np.ceil(3 * L2_BYTES / (3 * M * K + 4 * M))))
+        qs = [(t["x"] if i == 0 else torch.roll(t["x"], shifts=i, dims=0).contiguous(), torch.empty_like(t["ws_xq"]),
+               torch.empty_like(t["ws_scale_a"])) for i in range(nq)]
+        q = w8.w8a8_quantize_act_gelu if t["input_act"] == w8.ACT_GELU else w8.w8a8_quantize_act
+
+        def one(i):
+            x, xq, sa = qs[i % nq]
+            q(x, xq=xq, scale_a=sa, stream=stream)
+
+        ms = time_graph(one, stream, dev, nq * max(1, 10 // nq), 5)
+        del qs
+        return ms, nq
+
     for l in blk.layers:
         t = L[l.name]
-        qms = graph_ms(lambda i, t=t: quantize(t))
+        qms, nq = quantize_rotating_ms(t, l.K)
         lms = graph_ms(lambda i, t=t: linear(t))
         qbytes = 3 * M * l.K + 4 * M
         ops = 2.0 * M * l.N * l.K
-        comps[l.name] = {"N": l.N, "K": l.K, "input_act": l.act or "none", "gemm_ms_live": gemm_ms[l.name],
+        comps[l.name] = {"N": l.N, "K": l.K, "input_act": l.act or "none", "quantizer_rotation": nq,
+                         "gemm_ms_live": gemm_ms[l.name],
                          "gemm_tops_live": ops / (gemm_ms[l.name] * 1e-3) / 1e12,
                          "linear_ms": lms, "quantizer_ms": qms, "quantizer_gbs": qbytes / (qms * 1e-3) / 1e9,
                          "quantizer_frac_of_measured_hbm": qbytes / (qms * 1e-3) / 1e9 / peaks["hbm_gbs"],

@@ -149,6 +149,12 @@ W8A8_API w8a8_status w8a8_linear(const void* x, const int8_t* wq, const float* s
  * launch); if the device cannot guarantee that, the call fails with
  * W8A8_ERR_LAUNCH and nothing runs.  Results are bit-identical to
  * w8a8_linear.
+ * Performance: SLOWER than w8a8_linear on every DiT shape measured on B200
+ * (back to back, e.g. 4096 x 12288 x 3072: 132 us against 114 us; the long-K
+ * 9216 x 3072 x 12288: 313 against 289): only the GEMM's 8 epilogue warps
+ * per CTA can quantize, where the standalone quantizer runs 28 warps per
+ * SM.  Kept as the measured alternative placement of the quantizer; use
+ * w8a8_linear.
  */
 W8A8_API w8a8_status w8a8_linear_fused(const void* x, const int8_t* wq, const float* scale_w, const void* bias,
                                        void* out, int8_t* ws_xq, float* ws_scale_a, uint32_t* ws_sync,

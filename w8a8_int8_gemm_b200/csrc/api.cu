@@ -23,6 +23,7 @@ struct DeviceInfo {
   bool valid = false;
   bool supported = false;
   int sms = 0;
+  int64_t l2_bytes = 0;
 };
 
 constexpr int kMaxDevices = 64;
@@ -37,14 +38,16 @@ w8a8_status current_device(DeviceInfo* out) {
   std::lock_guard<std::mutex> lock(g_dev_mutex);
   DeviceInfo& d = g_devices[dev];
   if (!d.valid) {
-    int major = 0, minor = 0, sms = 0;
+    int major = 0, minor = 0, sms = 0, l2 = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess) {
       return W8A8_ERR_CUDA;
     }
     d.supported = (major == 10 && minor == 0);
     d.sms = sms;
+    d.l2_bytes = l2;
     d.valid = true;
   }
   *out = d;
@@ -152,6 +155,7 @@ w8a8_status gemm_common(const int8_t* xq, const int8_t* wq, const float* scale_a
   a.out_kind = kind;
   a.elem = elem;
   a.timeout_ns = static_cast<uint64_t>(g_timeout_ns.load());
+  a.l2_bytes = dev.l2_bytes;
   a.overlap_prologue = overlap_prologue;
   GemmConfig c{cfg.block_m, cfg.block_n, cfg.stages, cfg.grid, cfg.raster_group};
   return from_cuda(launch_gemm(a, c, stream));
@@ -314,6 +318,7 @@ w8a8_status w8a8_linear_fused(const void* x, const int8_t* wq, const float* scal
   a.K = K;
   a.out_kind = GemmOut::kBf16Dequant;
   a.timeout_ns = static_cast<uint64_t>(g_timeout_ns.load());
+  a.l2_bytes = dev.l2_bytes;
   a.fused = true;
   a.x = x;
   a.ldx = K;

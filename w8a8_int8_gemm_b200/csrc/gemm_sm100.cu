@@ -85,6 +85,11 @@ struct Params {
   const __nv_bfloat16* bias;
   uint64_t timeout_ns;
   int* err;  // device error word
+  // L2 policy of the A operand (the activations): evict_last, like B, while
+  // A is small enough to stay in L2 beside B; evict_first when A alone is
+  // more than half of L2 (long-K layers: A is then streamed once per tile
+  // row and would push B out, which every tile row reads again).
+  int a_evict_first;
   // Fused linear layer only: the bf16 activations, the workspace the kernel
   // quantizes them into (xq is also the A operand of tm_a), and the
   // row-block counters ([m_tiles] blocks + 1 CTA counter, zero on entry).
@@ -276,8 +281,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     int ready_mb = -1;  // fused layer: the last row block known to be quantized
     // Both operands are read again by other tiles: keep them in L2 ahead of
-    // the streamed output.
+    // the streamed output -- B always; A unless it is too large to stay.
     const uint64_t keep = l2_policy_evict_last();
+    const uint64_t a_pol = p.a_evict_first ? l2_policy_evict_first() : keep;
     for (int item = unit; ok && item < p.work_items; item += num_units) {
       int mb, nb, hb;
       item_coords(item, p, mb, nb, hb);
@@ -299,19 +305,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (leader) mbar_arrive_expect_tx(&full[stage], tx_bytes);
             tma_load_3d_pair_hint(sB + stage * kB, map_b, bar, 0, b_row, 2 * kb, keep);
             if (fills == 0) pdl_wait_prerequisites();  // A may be written by the kernel before this one
-            tma_load_3d_pair_hint(sA + stage * kA, &tm_a, bar, 0, a_row, 2 * kb, keep);
+            tma_load_3d_pair_hint(sA + stage * kA, &tm_a, bar, 0, a_row, 2 * kb, a_pol);
           } else if constexpr (PAIR) {
             const uint32_t bar = map_to_cta(smem_u32(&full[stage]), 0u);
             if (leader) mbar_arrive_expect_tx(&full[stage], tx_bytes);
             tma_load_2d_pair_hint(sB + stage * kB, map_b, bar, kb * kBlockK, b_row, keep);
             if (fills == 0) pdl_wait_prerequisites();  // A may be written by the kernel before this one
-            tma_load_2d_pair_hint(sA + stage * kA, &tm_a, bar, kb * kBlockK, a_row, keep);
+            tma_load_2d_pair_hint(sA + stage * kA, &tm_a, bar, kb * kBlockK, a_row, a_pol);
           } else {
             mbar_arrive_expect_tx(&full[stage], tx_bytes);
             tma_load_2d_hint(sB + stage * kB, map_b, &full[stage], kb * kBlockK, b_row, keep);
             if constexpr (!FUSE) {
               if (fills == 0) pdl_wait_prerequisites();  // A may be written by the kernel before this one
-              tma_load_2d_hint(sA + stage * kA, &tm_a, &full[stage], kb * kBlockK, a_row, keep);
+              tma_load_2d_hint(sA + stage * kA, &tm_a, &full[stage], kb * kBlockK, a_row, a_pol);
             }
           }
         }
@@ -329,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           // After a failed wait the load is still issued (its data is
           // discarded): the stage's barrier completes and teardown drains it.
-          if (lane == 0) tma_load_2d_hint(sA + stage * kA, &tm_a, &full[stage], kb * kBlockK, a_row, keep);
+          if (lane == 0) tma_load_2d_hint(sA + stage * kA, &tm_a, &full[stage], kb * kBlockK, a_row, a_pol);
           if (!ok) {
             __syncwarp();
             ++fills;
@@ -751,6 +757,7 @@ cudaError_t launch_typed(const GemmArgs& a, const GemmConfig& cfg, cudaStream_t 
   p.bias = static_cast<const __nv_bfloat16*>(a.bias);
   p.timeout_ns = a.timeout_ns;
   p.err = nullptr;
+  p.a_evict_first = a.M * a.K > a.l2_bytes / 2 ? 1 : 0;
   p.x = static_cast<const __nv_bfloat16*>(a.x);
   p.ldx = a.ldx;
   p.xq_out = const_cast<int8_t*>(a.xq);

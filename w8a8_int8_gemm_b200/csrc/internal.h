@@ -37,6 +37,7 @@ struct GemmArgs {
   GemmOut out_kind;
   GemmElem elem = GemmElem::kInt8;
   uint64_t timeout_ns;
+  int64_t l2_bytes = 0;  // L2 size of the device (chooses the A operand's cache policy)
   // The fused linear layer: quantize x [M, K] (bf16, row stride ldx) into
   // xq / scale_a inside the GEMM kernel (xq and scale_a are then outputs);
   // sync is the zeroed row-block counter workspace (linear_sync_words(M)).

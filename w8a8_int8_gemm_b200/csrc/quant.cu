@@ -271,10 +271,38 @@ __device__ __forceinline__ uint32_t lut_pair(const uint16_t* table, uint32_t w) 
   return r;
 }
 
+__device__ __forceinline__ void st_cluster_u16(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u16 [%0], %1;" ::"r"(cluster_addr), "h"(static_cast<unsigned short>(v))
+               : "memory");
+}
+
+// The bf16 inputs whose GELU has no closed form and takes the binary64
+// evaluation (see qrow::gelu_bf16_bits): 0x3580..0x407F (2^-20 < h < 4),
+// 0xB580..0xC12F (-11 < h < -2^-20), and the infinities and NaNs
+// 0x7F80..0x7FFF, 0xFF80..0xFFFF -- 6064 patterns, all runs of 8 aligned.
+constexpr int kGeluSlowPatterns = (0x4080 - 0x3580) + (0xC130 - 0xB580) + 128 + 128;
+
+__device__ __forceinline__ uint32_t gelu_slow_pattern(int f) {
+  if (f < 0x4080 - 0x3580) return 0x3580u + static_cast<uint32_t>(f);
+  f -= 0x4080 - 0x3580;
+  if (f < 0xC130 - 0xB580) return 0xB580u + static_cast<uint32_t>(f);
+  f -= 0xC130 - 0xB580;
+  return (f < 128 ? 0x7F80u : 0xFF80u - 128u) + static_cast<uint32_t>(f);
+}
+
+__device__ __forceinline__ bool gelu_slow_run(uint32_t u) {
+  return (u >= 0x3580u && u < 0x4080u) || (u >= 0xB580u && u < 0xC130u) || (u >= 0x7F80u && u < 0x8000u) ||
+         u >= 0xFF80u;
+}
+
 // The table of bf16_rne(GELU(h)) for every bf16 bit pattern h, built by a
-// cluster: this CTA computes 65536 / cluster consecutive entries (8 per
-// call of gelu_bf16x8) and stores each 16-byte run into the table of every CTA
-// of the cluster.  The caller synchronises the cluster before any lookup.
+// cluster and stored into the shared memory of every CTA of it.  The 59472
+// entries with a closed form go first, this CTA taking 65536 / cluster
+// consecutive patterns as 16-byte runs of 8 (one call of gelu_bf16x8 each);
+// the 6064 binary64 evaluations are then dealt one per thread across the
+// whole cluster (they lie in a few contiguous ranges, which whole runs would
+// leave to one or two CTAs) and stored entry by entry.  The caller
+// synchronises the cluster before any lookup.
 __device__ __forceinline__ void build_gelu_table(uint16_t* table, int cluster) {
   const uint32_t rank = cluster_ctarank();
   const int per_cta = 65536 / cluster;
@@ -282,10 +310,17 @@ __device__ __forceinline__ void build_gelu_table(uint16_t* table, int cluster) {
   for (int e = static_cast<int>(rank) * per_cta + static_cast<int>(threadIdx.x) * 8;
        e < static_cast<int>(rank + 1) * per_cta; e += static_cast<int>(blockDim.x) * 8) {
     const uint32_t u = static_cast<uint32_t>(e);
+    if (gelu_slow_run(u)) continue;
     const uint4 pats = make_uint4(u | ((u + 1) << 16), (u + 2) | ((u + 3) << 16), (u + 4) | ((u + 5) << 16),
                                   (u + 6) | ((u + 7) << 16));
     const uint4 g = qrow::gelu_bf16x8(pats);
     for (int r = 0; r < cluster; ++r) st_cluster_v4(map_to_cta(table_addr + 2u * u, static_cast<uint32_t>(r)), g);
+  }
+  const int stride = cluster * static_cast<int>(blockDim.x);
+  for (int f = static_cast<int>(rank) + cluster * static_cast<int>(threadIdx.x); f < kGeluSlowPatterns; f += stride) {
+    const uint32_t u = gelu_slow_pattern(f);
+    const uint32_t g = qrow::gelu_bf16_bits(u);
+    for (int r = 0; r < cluster; ++r) st_cluster_u16(map_to_cta(table_addr + 2u * u, static_cast<uint32_t>(r)), g);
   }
 }
 

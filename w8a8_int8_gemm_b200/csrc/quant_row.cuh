@@ -64,7 +64,25 @@ __device__ __forceinline__ uint64_t neg(uint64_t a) { return a ^ 0x8000000080000
 // value is within far less than 2^-40 (relative) of the exact function, so
 // the result is its correctly rounded bf16 value except where that lies
 // nearer a rounding boundary than this error.
+//
+// Outside -11 < h < 4 and away from 0 the function is a closed form, taken
+// without the binary64 evaluation (each equal to it for every bf16 input,
+// which the exhaustive comparison with the CPU oracle checks):
+//   h >= 4:        1 + exp(-2u) < 1 + 2^-15, so the result is h itself;
+//   h <= -11:      |gelu(h)| is below half the least bf16 subnormal: -0;
+//   |h| <= 2^-20:  gelu(h) = h/2 + 0.399 h^2 + ..., the h^2 term far below
+//                  binary64's resolution of h/2, so the result is
+//                  bf16_rne(h/2) (h/2 formed exactly in binary32).
+// That leaves under 6000 of the 65536 bf16 inputs for the binary64 path.
 __device__ __forceinline__ uint32_t gelu_bf16_bits(uint32_t hb) {
+  const uint32_t m = hb & 0x7FFFu;
+  if (m <= 0x3580u) {  // |h| <= 2^-20 (zeros included)
+    return __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(__uint_as_float(hb << 16), 0.5f)));
+  }
+  if (m < 0x7F80u) {  // finite
+    if (hb < 0x8000u && m >= 0x4080u) return hb;        // h >= 4
+    if (hb >= 0x8000u && m >= 0x4130u) return 0x8000u;  // h <= -11
+  }
   const double h = static_cast<double>(__uint_as_float(hb << 16));
   const double h3 = __dmul_rn(__dmul_rn(h, h), h);
   const double inner = __dadd_rn(h, __dmul_rn(0.044715, h3));
