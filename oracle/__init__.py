@@ -15,8 +15,9 @@ bf16 output), is stated in the C file's header.
 
 Every function is pinned by the CPU tests to something other than itself
 (numpy's float32 division and rint, numpy's int64 matmul, torch's bf16
-conversion, hand-worked examples, closed forms and invariants).  No
-function is "parity unpinned".
+conversion, hand-worked examples, closed forms and invariants; GELU to the
+correctly rounded bf16 value of the exact function in 60-digit decimal
+arithmetic on every bf16 input).  No function is "parity unpinned".
 """
 from __future__ import annotations
 

@@ -56,3 +56,20 @@ def test_traffic_files_only_count_for_the_sources_they_were_taken_on(monkeypatch
     assert b.ncu_traffic(workload, kind)["dram_bytes_per_launch"] == rec["dram_bytes_per_launch"]
     monkeypatch.setattr(b, "gemm_source_hash", lambda: "0" * 16)
     assert b.ncu_traffic(workload, kind) is None
+
+
+def test_roofline_peak_follows_the_timed_region():
+    """The tensor peak a roofline fraction is taken against: twice the
+    measured bf16 figure, the burst one for a timed region under a second,
+    the sustained one for a second or more; the other fractions beside it."""
+    b = _bench_module()
+    peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0, "source": "measured"}
+    short = b.tensor_peak(peaks, 2.4)
+    assert short["kind"] == "burst" and short["peak"] == 3200.0
+    long_ = b.tensor_peak(peaks, 1500.0)
+    assert long_["kind"] == "sustained" and long_["peak"] == 2800.0
+    assert b.tensor_peak(peaks, 1000.0)["kind"] == "sustained"
+    det = short["detail"](1600.0)
+    assert det["frac_of_burst_peak"] == 0.5 and det["frac_of_sustained_peak"] == 1600.0 / 2800.0
+    assert abs(det["frac_of_spec_4p5"] - 1600.0 / 4500.0) < 1e-12
+    assert "2.4 ms" in det["peak_source"] and "burst" in det["peak_source"]

@@ -26,7 +26,7 @@ import torch
 import oracle
 import workloads
 from tests.oracle_pins import edge_rows
-from tests.util import bf16_bits_to_torch, bf16_ulp_diff, is_nan_bits, sample_rows, torch_bf16_to_bits
+from tests.util import bf16_bits_to_torch, bf16_ulp_diff, is_nan_bits, row_chunks, torch_bf16_to_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -309,26 +309,34 @@ def test_linear_fp8(w8, M, N, K):
     assert _within(got, want, vb).all()
 
 
-def test_linear_fp8_mlp_up_1024_sampled(w8):
-    """1024px MLP up-projection, 4096 x 12288 x 3072: the whole launch runs;
-    the oracle checks the weight codes, and sampled rows end to end."""
+def test_linear_fp8_mlp_up_1024_every_row(w8):
+    """1024px MLP up-projection, 4096 x 12288 x 3072, in the launch
+    configuration the benchmark uses: the weight codes and scales, every
+    token's codes and scale bit-exact; every output row within one bf16 ulp
+    plus the propagated fp32-summation bound of the oracle's exact sum (its
+    GEMM in row chunks)."""
     wl = workloads.WORKLOADS["mlp_up_1024"]
     d = workloads.make(wl)
     dev = torch.device("cuda")
     wq, sw = w8.w8a8_quantize_weight_fp8(torch.from_numpy(d["w"]).to(dev))
-    out = w8.w8a8_linear_fp8(bf16_bits_to_torch(d["x"], dev), wq, sw, bf16_bits_to_torch(d["bias"], dev))
+    xq = torch.empty((wl.M, wl.K), dtype=torch.uint8, device=dev)
+    sa = torch.empty((wl.M,), dtype=torch.float32, device=dev)
+    out = w8.w8a8_linear_fp8(bf16_bits_to_torch(d["x"], dev), wq, sw, bf16_bits_to_torch(d["bias"], dev),
+                             ws_xq=xq, ws_scale_a=sa)
     torch.cuda.synchronize()
     wq_want, sw_want = oracle.quantize_weight_fp8(d["w"])
     assert np.array_equal(wq.cpu().numpy(), wq_want) and np.array_equal(sw.cpu().numpy(), sw_want)
-    rows = sample_rows(wl.M, 40, 29)
-    xq_r, sa_r = oracle.quantize_act_fp8(d["x"][rows])
-    exact = oracle.gemm_fp8(xq_r, wq_want)
-    want = oracle.epilogue_fp8(exact, sa_r, sw_want, d["bias"])
-    vb = (wl.K - 1) * U23 * _abs_sum(xq_r, wq_want) * sa_r[:, None].astype(np.float64) * sw_want[None, :]
-    got = torch_bf16_to_bits(out)[rows]
-    assert not is_nan_bits(got).any()
-    ok = _within(got, want, vb)
-    assert ok.all(), (int((~ok).sum()), int(bf16_ulp_diff(got, want).max()))
+    xq_want, sa_want = oracle.quantize_act_fp8(d["x"])
+    assert np.array_equal(xq.cpu().numpy(), xq_want) and np.array_equal(sa.cpu().numpy(), sa_want)
+    got_all = torch_bf16_to_bits(out)
+    assert not is_nan_bits(got_all).any()
+    for rows in row_chunks(wl.M):
+        exact = oracle.gemm_fp8(xq_want[rows], wq_want)
+        want = oracle.epilogue_fp8(exact, sa_want[rows], sw_want, d["bias"])
+        vb = (wl.K - 1) * U23 * _abs_sum(xq_want[rows], wq_want) * sa_want[rows, None].astype(np.float64) * \
+            sw_want[None, :]
+        ok = _within(got_all[rows], want, vb)
+        assert ok.all(), (rows, int((~ok).sum()), int(bf16_ulp_diff(got_all[rows], want).max()))
 
 
 def test_fp8_empty_and_errors(w8):
