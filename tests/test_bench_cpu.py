@@ -73,3 +73,22 @@ def test_roofline_peak_follows_the_timed_region():
     assert det["frac_of_burst_peak"] == 0.5 and det["frac_of_sustained_peak"] == 1600.0 / 2800.0
     assert abs(det["frac_of_spec_4p5"] - 1600.0 / 4500.0) < 1e-12
     assert "2.4 ms" in det["peak_source"] and "burst" in det["peak_source"]
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    """Launched as the round-end scaling run launches it (torchrun, two ranks
+    on this host), the reference arm's rank 0 alone runs and prints its one
+    line; the other rank exits 0 without work."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--gpus", "2", "--workload", "tiny", "--steps", "3", "--warmup", "3"]
+    out = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1, out.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
