@@ -853,6 +853,27 @@ def measure_config(w8, wl, dev, stream, peaks: dict, cpu: bool) -> dict:
             continue
         ms = time_graph(fn, stream, dev, n, 3)
         res[fn.__name__ + "_us"] = None if ms is None else 1e3 * ms
+    # The paper's accuracy metric on this configuration: the output of one
+    # fresh call on the first buffer set against the float64 product on 64
+    # sampled rows (of the unquantized operands for bf16 inputs; of the
+    # dequantized codes where int8 codes are given), and NaNs in the whole
+    # output.
+    s0 = sets[0]
+    (linear if linear_kind else gemm)(0)
+    torch.cuda.synchronize(dev)
+    rows = torch.linspace(0, M - 1, min(64, M), device=dev).round().long()
+    b64 = bias.double()
+    if linear_kind:
+        ref = s0["x"][rows].double() @ torch.from_numpy(d["w"]).to(dev).double().t() + b64
+    else:
+        ref = (s0["xq"][rows].double() * s0["sa"][rows, None].double()) @ (
+            s0["wq"].double() * sw[:, None].double()).t() + b64
+    y = s0["out"][rows].double()
+    res["accuracy"] = {"cosine_vs_fp64": float((y * ref).sum() / (y.norm() * ref.norm())),
+                       "max_rel_err_vs_fp64": float(((y - ref).abs().max() / ref.abs().max())),
+                       "nan_outputs": int(torch.isnan(s0["out"]).sum()),
+                       "against": "unquantized operands" if linear_kind else "dequantized int8 codes",
+                       "rows": int(rows.numel())}
     if cpu:
         work = OracleWork(wl, pool_rows=256)
         rows, cols = size_sample(work, 1.5)

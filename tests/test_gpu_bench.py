@@ -45,3 +45,25 @@ def test_native_arm_json_line():
     assert e["h2d_bytes_per_step"] == 4096 * 3072 * 2 and e["d2h_bytes_per_step"] == 4096 * 12288 * 2
     assert 0 < e["value"] < d["value"]
     assert "sm_mhz" in d["clocks"] and "reasons" in d["clocks"]
+
+
+def test_native_arm_per_config_table():
+    """The per-configuration table of the default bench line: every DiT
+    layer shape timed, with the paper's accuracy metric beside it (cosine
+    similarity against the float64 product, no NaN in the output)."""
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--steps", "4", "--warmup", "3", "--e2e-steps", "0",
+           "--no-cpu-baseline"]
+    out = subprocess.run(cmd, capture_output=True, text=True, timeout=1200, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-3000:]
+    d = json.loads([l for l in out.stdout.splitlines() if l.strip().startswith("{")][-1])
+    rows = d["per_config"]["configs"]
+    assert [r["workload"] for r in rows] == ["qkv_768", "mlp_up_1024", "mlp_down_1024", "sweep_qkv", "sweep_out",
+                                             "sweep_up", "sweep_down"]
+    for r in rows:
+        assert r["gemm_us"] > 0 and r["gemm_tops"] > 0, r["workload"]
+        acc = r["accuracy"]
+        assert acc["nan_outputs"] == 0, r["workload"]
+        # with x20 outlier channels (MLP up) the per-token quantization itself costs ~1e-3 of cosine
+        assert acc["cosine_vs_fp64"] > (0.99 if acc["against"] == "unquantized operands" else 0.9999), r
+        if r["workload"] != "mlp_down_1024":
+            assert r["linear_us"] > 0 and r["quant_gbs"] > 0, r["workload"]
