@@ -205,6 +205,18 @@ w8a8_status check_linear_io(const void* x, const int8_t* wq, const float* scale_
   return W8A8_OK;
 }
 
+// check_linear_io plus the caller's workspaces (non-null, 16-byte aligned):
+// every check of a w8a8_linear-style call, before any CUDA call.
+w8a8_status check_linear_call(const void* x, const int8_t* wq, const float* scale_w, const void* bias,
+                              const void* out, const void* ws_xq, const float* ws_scale_a, int64_t M, int64_t N,
+                              int64_t K) {
+  w8a8_status st = check_linear_io(x, wq, scale_w, bias, out, M, N, K);
+  if (st != W8A8_OK || M == 0 || N == 0) return st;
+  if (ws_xq == nullptr || ws_scale_a == nullptr) return W8A8_ERR_INVALID_ARG;
+  if (!aligned16(ws_xq) || !aligned16(ws_scale_a)) return W8A8_ERR_ALIGNMENT;
+  return W8A8_OK;
+}
+
 // W8A8_OK if the current device is supported (sm_100), from the cached
 // device properties.
 w8a8_status check_current_device() {
@@ -272,17 +284,8 @@ w8a8_status w8a8_gemm_i32_ex(const int8_t* xq, const int8_t* wq, int32_t* acc, i
 w8a8_status w8a8_linear(const void* x, const int8_t* wq, const float* scale_w, const void* bias, void* out,
                         int8_t* ws_xq, float* ws_scale_a, int64_t M, int64_t N, int64_t K, w8a8_stream_t stream) {
   // Validate the whole call before launching its first kernel.
-  w8a8_status st = check_gemm_shape(M, N, K);
-  if (st != W8A8_OK) return st;
-  if (M == 0 || N == 0) return W8A8_OK;
-  if (x == nullptr || wq == nullptr || scale_w == nullptr || out == nullptr || ws_xq == nullptr ||
-      ws_scale_a == nullptr) {
-    return W8A8_ERR_INVALID_ARG;
-  }
-  if (!aligned16(x) || !aligned16(wq) || !aligned16(scale_w) || !aligned16(bias) || !aligned16(out) ||
-      !aligned16(ws_xq) || !aligned16(ws_scale_a)) {
-    return W8A8_ERR_ALIGNMENT;
-  }
+  w8a8_status st = check_linear_call(x, wq, scale_w, bias, out, ws_xq, ws_scale_a, M, N, K);
+  if (st != W8A8_OK || M == 0 || N == 0) return st;
   st = w8a8_quantize_act(x, M, K, K, ws_xq, K, ws_scale_a, stream);
   if (st != W8A8_OK) return st;
   return gemm_common(ws_xq, wq, ws_scale_a, scale_w, bias, out, M, N, K, nullptr, GemmOut::kBf16Dequant,
@@ -292,17 +295,10 @@ w8a8_status w8a8_linear(const void* x, const int8_t* wq, const float* scale_w, c
 w8a8_status w8a8_linear_fused(const void* x, const int8_t* wq, const float* scale_w, const void* bias, void* out,
                               int8_t* ws_xq, float* ws_scale_a, uint32_t* ws_sync, int64_t M, int64_t N, int64_t K,
                               w8a8_stream_t stream) {
-  w8a8_status st = check_gemm_shape(M, N, K);
-  if (st != W8A8_OK) return st;
-  if (M == 0 || N == 0) return W8A8_OK;
-  if (x == nullptr || wq == nullptr || scale_w == nullptr || out == nullptr || ws_xq == nullptr ||
-      ws_scale_a == nullptr || ws_sync == nullptr) {
-    return W8A8_ERR_INVALID_ARG;
-  }
-  if (!aligned16(x) || !aligned16(wq) || !aligned16(scale_w) || !aligned16(bias) || !aligned16(out) ||
-      !aligned16(ws_xq) || !aligned16(ws_scale_a) || !aligned16(ws_sync)) {
-    return W8A8_ERR_ALIGNMENT;
-  }
+  w8a8_status st = check_linear_call(x, wq, scale_w, bias, out, ws_xq, ws_scale_a, M, N, K);
+  if (st != W8A8_OK || M == 0 || N == 0) return st;
+  if (ws_sync == nullptr) return W8A8_ERR_INVALID_ARG;
+  if (!aligned16(ws_sync)) return W8A8_ERR_ALIGNMENT;
   DeviceInfo dev;
   if ((st = current_device(&dev)) != W8A8_OK) return st;
   const w8a8_gemm_config cfg = select(M, N, K, dev.sms, /*allow_pair=*/false);
@@ -369,17 +365,9 @@ w8a8_status w8a8_gemm_fp8_f32(const uint8_t* xq, const uint8_t* wq, float* acc, 
 w8a8_status w8a8_linear_fp8(const void* x, const uint8_t* wq, const float* scale_w, const void* bias, void* out,
                             uint8_t* ws_xq, float* ws_scale_a, int64_t M, int64_t N, int64_t K,
                             w8a8_stream_t stream) {
-  w8a8_status st = check_gemm_shape(M, N, K);
-  if (st != W8A8_OK) return st;
-  if (M == 0 || N == 0) return W8A8_OK;
-  if (x == nullptr || wq == nullptr || scale_w == nullptr || out == nullptr || ws_xq == nullptr ||
-      ws_scale_a == nullptr) {
-    return W8A8_ERR_INVALID_ARG;
-  }
-  if (!aligned16(x) || !aligned16(wq) || !aligned16(scale_w) || !aligned16(bias) || !aligned16(out) ||
-      !aligned16(ws_xq) || !aligned16(ws_scale_a)) {
-    return W8A8_ERR_ALIGNMENT;
-  }
+  w8a8_status st = check_linear_call(x, reinterpret_cast<const int8_t*>(wq), scale_w, bias, out, ws_xq, ws_scale_a,
+                                     M, N, K);
+  if (st != W8A8_OK || M == 0 || N == 0) return st;
   st = w8a8_quantize_act_fp8(x, M, K, K, ws_xq, K, ws_scale_a, stream);
   if (st != W8A8_OK) return st;
   return gemm_common(reinterpret_cast<const int8_t*>(ws_xq), reinterpret_cast<const int8_t*>(wq), ws_scale_a,
@@ -409,17 +397,8 @@ w8a8_status w8a8_gelu(const void* h, int64_t M, int64_t K, int64_t ldh, void* g,
 w8a8_status w8a8_linear_gelu(const void* h, const int8_t* wq, const float* scale_w, const void* bias, void* out,
                              int8_t* ws_xq, float* ws_scale_a, int64_t M, int64_t N, int64_t K,
                              w8a8_stream_t stream) {
-  w8a8_status st = check_gemm_shape(M, N, K);
-  if (st != W8A8_OK) return st;
-  if (M == 0 || N == 0) return W8A8_OK;
-  if (h == nullptr || wq == nullptr || scale_w == nullptr || out == nullptr || ws_xq == nullptr ||
-      ws_scale_a == nullptr) {
-    return W8A8_ERR_INVALID_ARG;
-  }
-  if (!aligned16(h) || !aligned16(wq) || !aligned16(scale_w) || !aligned16(bias) || !aligned16(out) ||
-      !aligned16(ws_xq) || !aligned16(ws_scale_a)) {
-    return W8A8_ERR_ALIGNMENT;
-  }
+  w8a8_status st = check_linear_call(h, wq, scale_w, bias, out, ws_xq, ws_scale_a, M, N, K);
+  if (st != W8A8_OK || M == 0 || N == 0) return st;
   st = w8a8_quantize_act_gelu(h, M, K, K, ws_xq, K, ws_scale_a, stream);
   if (st != W8A8_OK) return st;
   return gemm_common(ws_xq, wq, ws_scale_a, scale_w, bias, out, M, N, K, nullptr, GemmOut::kBf16Dequant,

@@ -33,23 +33,10 @@ struct w8a8_chain_st {
 
 namespace {
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-// The checks w8a8_linear makes, before any CUDA call.
+// The checks w8a8_linear makes, before any CUDA call, and the layer's input step.
 w8a8_status check_layer(const w8a8_linear_desc& l) {
-  if (l.M < 0 || l.N < 0 || l.K < 16 || l.K > 133144 || l.K % 16 != 0 || l.N % 8 != 0) return W8A8_ERR_INVALID_ARG;
-  if (l.M > 2147483647 || l.N > 2147483647) return W8A8_ERR_INVALID_ARG;
   if (l.input_act != W8A8_ACT_NONE && l.input_act != W8A8_ACT_GELU) return W8A8_ERR_INVALID_ARG;
-  if (l.M == 0 || l.N == 0) return W8A8_OK;
-  if (l.x == nullptr || l.wq == nullptr || l.scale_w == nullptr || l.out == nullptr || l.ws_xq == nullptr ||
-      l.ws_scale_a == nullptr) {
-    return W8A8_ERR_INVALID_ARG;
-  }
-  if (!aligned16(l.x) || !aligned16(l.wq) || !aligned16(l.scale_w) || !aligned16(l.bias) || !aligned16(l.out) ||
-      !aligned16(l.ws_xq) || !aligned16(l.ws_scale_a)) {
-    return W8A8_ERR_ALIGNMENT;
-  }
-  return W8A8_OK;
+  return w8a8::check_linear_call(l.x, l.wq, l.scale_w, l.bias, l.out, l.ws_xq, l.ws_scale_a, l.M, l.N, l.K);
 }
 
 }  // namespace

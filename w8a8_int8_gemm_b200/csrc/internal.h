@@ -88,6 +88,10 @@ cudaError_t launch_selftest_wait(uint64_t timeout_ns, cudaStream_t stream);
 w8a8_status check_linear_io(const void* x, const int8_t* wq, const float* scale_w, const void* bias,
                             const void* out, int64_t M, int64_t N, int64_t K);
 w8a8_status check_current_device();
+// check_linear_io plus the non-null, 16-byte aligned workspaces ws_xq and ws_scale_a.
+w8a8_status check_linear_call(const void* x, const int8_t* wq, const float* scale_w, const void* bias,
+                              const void* out, const void* ws_xq, const float* ws_scale_a, int64_t M, int64_t N,
+                              int64_t K);
 
 // Synchronizes the current device and reads (optionally clears) the device
 // error word written by timed-out waits.
